@@ -1,0 +1,93 @@
+"""Seeded synthetic inputs shared by the tests, the smoke check and the bench.
+
+This module only draws random numbers and casts them; it holds none of the
+attention arithmetic, so both the CUDA path and the CPU oracle can be fed from
+it without sharing any of the method.
+
+Recipe (the same for every workload): a CPU ``torch.Generator`` seeded with
+``seed`` draws float32 standard normals of shape [B, N, H, d] in the order
+Q, K, V, dO.  For the long-sequence workload a further ``randperm(N)`` from the
+same generator picks floor(frac * N) sequence positions whose K rows (all
+batches and heads) are multiplied by ``spike`` in float32, which forces large
+jumps of the running row maximum in the online softmax.  The tensors are then
+cast to the working dtype with round-to-nearest-even.
+"""
+
+from __future__ import annotations
+
+import dataclasses
+import math
+
+import torch
+
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    """One attention problem: shapes, dtype, masks and which passes run."""
+
+    name: str
+    B: int
+    H: int
+    N: int
+    d: int
+    dtype: str = "bf16"           # "bf16" or "fp32"
+    causal: tuple = (False,)      # the mask settings the workload covers
+    backward: bool = False        # True when dQ, dK, dV are part of it
+    spike_frac: float = 0.0       # fraction of K rows scaled by ``spike``
+    spike: float = 3.0
+    seed: int = 0
+
+    def flops_fwd(self, causal: bool) -> float:
+        """4*B*H*N^2*d, halved when causal (the usual attention count)."""
+        f = 4.0 * self.B * self.H * self.N * self.N * self.d
+        return f / 2 if causal else f
+
+
+# The five problem families the method is measured on.
+FP32_SMALL = Workload("fp32 fwd B1 H1 N256 d64", 1, 1, 256, 64, "fp32", (False,))
+BF16_FWD_N1K = Workload("bf16 fwd B4 H16 N1024 d64", 4, 16, 1024, 64, "bf16", (False, True))
+BF16_FWDBWD_N4K = Workload("bf16 fwd+bwd B2 H16 N4096 d128 causal", 2, 16, 4096, 128, "bf16",
+                           (True,), backward=True)
+BF16_FWDBWD_N16K = Workload("bf16 fwd+bwd B1 H32 N16384 d128 K-spike", 1, 32, 16384, 128, "bf16",
+                            (False, True), backward=True, spike_frac=0.01, spike=3.0)
+SWEEP = tuple(
+    Workload(f"bf16 fwd sweep B{b} H{h} N{n} d{d}", b, h, n, d, "bf16", (False, True))
+    for (b, h, n, d) in ((16, 16, 512, 64), (8, 16, 1024, 128), (4, 32, 2048, 128),
+                         (2, 32, 8192, 128), (1, 16, 32768, 128))
+)
+ALL = (FP32_SMALL, BF16_FWD_N1K, BF16_FWDBWD_N4K, BF16_FWDBWD_N16K) + SWEEP
+
+
+def torch_dtype(name: str) -> torch.dtype:
+    return {"bf16": torch.bfloat16, "fp32": torch.float32}[name]
+
+
+def make_inputs(B: int, N: int, H: int, d: int, *, seed: int = 0, dtype: str = "bf16",
+                spike_frac: float = 0.0, spike: float = 3.0, with_do: bool = True):
+    """Return CPU tensors (q, k, v, do) of shape [B, N, H, d] in ``dtype``.
+
+    ``do`` is None when ``with_do`` is False (it is still drawn, so Q, K, V
+    are the same either way).
+    """
+    g = torch.Generator(device="cpu").manual_seed(int(seed))
+    shape = (B, N, H, d)
+    q = torch.randn(shape, generator=g, dtype=torch.float32)
+    k = torch.randn(shape, generator=g, dtype=torch.float32)
+    v = torch.randn(shape, generator=g, dtype=torch.float32)
+    do = torch.randn(shape, generator=g, dtype=torch.float32)
+    if spike_frac > 0 and N > 0:
+        count = int(math.floor(spike_frac * N))
+        if count > 0:
+            idx = torch.randperm(N, generator=g)[:count]
+            k[:, idx] *= float(spike)
+    td = torch_dtype(dtype)
+    out = [t.to(td).contiguous() for t in (q, k, v, do)]
+    if not with_do:
+        out[3] = None
+    return tuple(out)
+
+
+def workload_inputs(w: Workload, *, with_do=None):
+    return make_inputs(w.B, w.N, w.H, w.d, seed=w.seed, dtype=w.dtype,
+                       spike_frac=w.spike_frac, spike=w.spike,
+                       with_do=w.backward if with_do is None else with_do)

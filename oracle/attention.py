@@ -1,0 +1,264 @@
+"""Plain fp64 CPU oracle for exact scaled-dot-product attention.
+
+TEST INFRASTRUCTURE ONLY.  Only the test suite, the smoke check in
+``__graft_entry__`` and the CPU-baseline leg of ``bench.py`` may import this
+module.  The product path (the CUDA library and its Python binding) never
+imports or calls it, and this module imports nothing from the product.
+
+What it computes, and where the pages define it
+-----------------------------------------------
+Sources (web pages on FlashAttention; cited by page title and section):
+
+* "Flash Attention" (karlkratz.de), sections "Tiling: Blockweise Berechnung im
+  schnellen Speicher", "Speicherbedarf und Laufzeitverhalten",
+  "Recomputation beim Rückwärtsdurchlauf".
+* "Flash Attention" (Ultralytics glossary), sections "Принцип работы Flash
+  Attention" (algorithm description and the PyTorch demonstration with its
+  printed error) and "Flash Attention и смежные понятия" (standard attention).
+
+Both pages state that the tiled method computes *exactly* standard attention
+(up to floating-point rounding), so the oracle is the plain definition written
+out, materialising the full score matrix S and probability matrix P per
+(batch, head) in float64:
+
+    S_ij  = scale * <q_i, k_j>            (-inf where j > i when causal)
+    m_i   = max_j S_ij
+    P_ij  = exp(S_ij - m_i) / sum_j exp(S_ij - m_i)
+    O_i   = sum_j P_ij v_j
+    LSE_i = m_i + ln sum_j exp(S_ij - m_i)          (natural log)
+
+Backward (the pages only say that score blocks are recomputed from Q, K, V;
+the gradient formulas are calculus on the definition above, with dO the
+incoming gradient of O and LSE treated as a non-differentiable side output):
+
+    dV = P^T dO
+    dP = dO V^T
+    D_i = sum_k dO_ik O_ik            (= sum_j P_ij dP_ij)
+    dS = P * (dP - D)                 (elementwise, D broadcast over j)
+    dQ = scale * dS K
+    dK = scale * dS^T Q
+
+Readings where the pages are silent (all recorded in the design notes):
+* one LSE per row in natural-log units replaces the "two numbers per row"
+  (running max and running sum) because P = exp(S - LSE) recovers both;
+* causal masking is top-left aligned (key j visible to query i iff j <= i),
+  the only reading with equal query and key lengths;
+* inputs are the exact values the GPU sees (bf16 or fp32 widened to fp64) and
+  ``scale`` is the fp32 value the GPU receives, widened.
+
+``blocked_forward_head`` restates the pages' online-softmax algorithm (key
+blocks streamed, running row max and sum, rescale when the max grows) and is
+used only to pin the oracle: blocked and full results must agree.
+
+Parity pins: every function here is pinned by ``tests/test_oracle.py``
+(closed forms, invariants, finite differences, the pages' worked example).
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+__all__ = [
+    "scores_head",
+    "probs_head",
+    "forward_head",
+    "forward_rows_head",
+    "backward_head",
+    "blocked_forward_head",
+    "forward",
+    "backward",
+]
+
+
+def _f64(x) -> np.ndarray:
+    a = np.asarray(x)
+    return a.astype(np.float64, copy=False)
+
+
+def scores_head(q, k, scale: float, causal: bool) -> np.ndarray:
+    """S = scale * Q K^T for one (batch, head), with the causal mask applied.
+
+    q: [Nq, d], k: [Nk, d].  Masked entries are -inf.  Query row i sits at
+    sequence position i (top-left alignment), so key j is hidden when j > i.
+    Standard attention as defined in "Flash Attention" (Ultralytics glossary),
+    "Flash Attention и смежные понятия" (the same operation with the full
+    score matrix written out).
+    """
+    q = _f64(q)
+    k = _f64(k)
+    s = float(scale) * (q @ k.T)
+    if causal:
+        nq, nk = s.shape
+        hidden = np.arange(nk)[None, :] > np.arange(nq)[:, None]
+        s = np.where(hidden, -np.inf, s)
+    return s
+
+
+def probs_head(s: np.ndarray):
+    """Row softmax of a score matrix.  Returns (P, LSE) with LSE natural-log.
+
+    A row whose entries are all -inf (no visible key) gets P = 0 and
+    LSE = -inf; with equal query and key lengths causal masking never
+    produces one.
+    """
+    m = np.max(s, axis=1, keepdims=True)
+    m_safe = np.where(np.isfinite(m), m, 0.0)
+    e = np.exp(s - m_safe)
+    l = np.sum(e, axis=1, keepdims=True)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        p = np.where(l > 0, e / np.where(l > 0, l, 1.0), 0.0)
+        lse = np.where(l[:, 0] > 0, m_safe[:, 0] + np.log(np.where(l[:, 0] > 0, l[:, 0], 1.0)), -np.inf)
+    return p, lse
+
+
+def forward_head(q, k, v, scale: float, causal: bool):
+    """O = softmax(scale Q K^T + mask) V and LSE for one (batch, head).
+
+    q, k, v: [N, d].  Returns O [N, d] float64 and LSE [N] float64.
+    Definition of the exact result the tiled kernel must reproduce:
+    "Flash Attention" (karlkratz.de), "Speicherbedarf und Laufzeitverhalten"
+    (same result, not an approximation).
+    """
+    s = scores_head(q, k, scale, causal)
+    p, lse = probs_head(s)
+    return p @ _f64(v), lse
+
+
+def forward_rows_head(q, k, v, rows, scale: float, causal: bool):
+    """Forward restricted to the query rows ``rows`` of one (batch, head).
+
+    A row of O and its LSE depend only on that query row and all of K and V,
+    so this is the definition evaluated on a subset of rows (used to check
+    large problems on sampled rows).
+    """
+    rows = np.asarray(rows, dtype=np.int64)
+    q = _f64(q)
+    k = _f64(k)
+    s = float(scale) * (q[rows] @ k.T)
+    if causal:
+        hidden = np.arange(k.shape[0])[None, :] > rows[:, None]
+        s = np.where(hidden, -np.inf, s)
+    p, lse = probs_head(s)
+    return p @ _f64(v), lse
+
+
+def backward_head(q, k, v, do, scale: float, causal: bool):
+    """Gradients (dQ, dK, dV) of O = attention(Q, K, V) given dO, one head.
+
+    Recomputes S and P from Q, K and V ("Flash Attention" (karlkratz.de),
+    "Recomputation beim Rückwärtsdurchlauf": the backward recomputes the
+    attention values instead of storing them).  Also returns D = rowsum(dO*O).
+    """
+    q = _f64(q)
+    k = _f64(k)
+    v = _f64(v)
+    do = _f64(do)
+    s = scores_head(q, k, scale, causal)
+    p, _ = probs_head(s)
+    o = p @ v
+    dv = p.T @ do
+    dp = do @ v.T
+    dvec = np.sum(do * o, axis=1)
+    ds = p * (dp - dvec[:, None])
+    dq = float(scale) * (ds @ k)
+    dk = float(scale) * (ds.T @ q)
+    return dq, dk, dv, dvec
+
+
+def blocked_forward_head(q, k, v, scale: float, causal: bool, block: int,
+                         tau: float = 0.0, dtype=np.float64):
+    """Online-softmax forward over key blocks, as the pages describe it.
+
+    Follows "Flash Attention" (Ultralytics glossary), "Принцип работы Flash
+    Attention": all query rows are held at once, key/value blocks stream past;
+    for each block the scores are formed, the running row maximum and running
+    row sum are updated, the partial output is rescaled when the maximum
+    grows, and the block's weighted values are added; finally the output is
+    divided by the running sum.  "Flash Attention" (karlkratz.de), "Tiling"
+    describes the same per-row pair (maximum, sum) and correction factor.
+
+    ``tau`` > 0 is the lazy variant: the reference maximum is only moved when
+    the new block maximum exceeds it by more than ``tau`` (natural-log units);
+    numerator and denominator share the same reference, so the result is the
+    same.  ``dtype`` selects the working precision (float64 for pins of the
+    exact result, float32 to reproduce the pages' fp32 demonstration).
+    Returns (O, LSE).
+    """
+    q = np.asarray(q, dtype=dtype)
+    k = np.asarray(k, dtype=dtype)
+    v = np.asarray(v, dtype=dtype)
+    n, d = q.shape
+    nk = k.shape[0]
+    sc = dtype(scale)
+    run_max = np.full((n, 1), -np.inf, dtype=dtype)
+    run_sum = np.zeros((n, 1), dtype=dtype)
+    acc = np.zeros((n, v.shape[1]), dtype=dtype)
+    rows = np.arange(n)[:, None]
+    for start in range(0, nk, block):
+        stop = min(start + block, nk)
+        s = (q @ k[start:stop].T) * sc
+        if causal:
+            cols = np.arange(start, stop)[None, :]
+            s = np.where(cols > rows, dtype(-np.inf), s)
+        blk_max = np.max(s, axis=1, keepdims=True)
+        cand = np.maximum(run_max, blk_max)
+        move = cand > run_max + dtype(tau) if tau > 0 else cand > run_max
+        new_max = np.where(move | ~np.isfinite(run_max), cand, run_max)
+        base = np.where(np.isfinite(new_max), new_max, dtype(0))
+        with np.errstate(invalid="ignore"):
+            corr = np.where(np.isfinite(run_max), np.exp(run_max - base), dtype(0))
+        e = np.exp(s - base)
+        run_sum = run_sum * corr + np.sum(e, axis=1, keepdims=True)
+        acc = acc * corr + e @ v[start:stop]
+        run_max = new_max
+    with np.errstate(divide="ignore", invalid="ignore"):
+        out = np.where(run_sum > 0, acc / np.where(run_sum > 0, run_sum, 1), 0)
+        lse = np.where(run_sum[:, 0] > 0,
+                       np.where(np.isfinite(run_max[:, 0]), run_max[:, 0], 0)
+                       + np.log(np.where(run_sum[:, 0] > 0, run_sum[:, 0], 1)), -np.inf)
+    return out.astype(dtype), lse.astype(dtype)
+
+
+def forward(Q, K, V, scale: float, causal: bool, heads=None):
+    """Batched forward over [B, N, H, d] tensors (numpy or CPU torch).
+
+    Returns O [B, N, H, d] and LSE [B, H, N] in float64.  ``heads`` restricts
+    the work to a list of (b, h) pairs; other entries are left as NaN.
+    """
+    Q, K, V = (_f64(_to_numpy(t)) for t in (Q, K, V))
+    b_, n_, h_, d_ = Q.shape
+    O = np.full((b_, n_, h_, V.shape[3]), np.nan)
+    LSE = np.full((b_, h_, n_), np.nan)
+    for (b, h) in (heads if heads is not None else _all_heads(b_, h_)):
+        o, lse = forward_head(Q[b, :, h], K[b, :, h], V[b, :, h], scale, causal)
+        O[b, :, h] = o
+        LSE[b, h] = lse
+    return O, LSE
+
+
+def backward(Q, K, V, dO, scale: float, causal: bool, heads=None):
+    """Batched backward over [B, N, H, d].  Returns dQ, dK, dV (float64)."""
+    Q, K, V, dO = (_f64(_to_numpy(t)) for t in (Q, K, V, dO))
+    shape = Q.shape
+    dQ = np.full(shape, np.nan)
+    dK = np.full(shape, np.nan)
+    dV = np.full(V.shape, np.nan)
+    for (b, h) in (heads if heads is not None else _all_heads(shape[0], shape[2])):
+        dq, dk, dv, _ = backward_head(Q[b, :, h], K[b, :, h], V[b, :, h], dO[b, :, h], scale, causal)
+        dQ[b, :, h] = dq
+        dK[b, :, h] = dk
+        dV[b, :, h] = dv
+    return dQ, dK, dV
+
+
+def _all_heads(nb, nh):
+    return [(b, h) for b in range(nb) for h in range(nh)]
+
+
+def _to_numpy(t):
+    if hasattr(t, "detach"):
+        t = t.detach()
+        if hasattr(t, "dtype") and str(t.dtype) == "torch.bfloat16":
+            t = t.float()
+        return t.cpu().numpy()
+    return np.asarray(t)

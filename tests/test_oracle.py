@@ -1,0 +1,387 @@
+"""Pins for the CPU oracle: checks against what the pages and the mathematics fix.
+
+None of these re-type the oracle's formulas; each compares it with something
+independent of it: closed-form outputs, invariants, the pages' worked example,
+central finite differences, or a library routine on a special case.  The
+mutation tests at the end plant plausible mistakes in copies of the oracle and
+check that at least one pin catches each.
+"""
+
+from __future__ import annotations
+
+import json
+import math
+import pathlib
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle import attention as A
+
+GOLDEN = pathlib.Path(__file__).parent / "golden"
+
+
+def _rand(shape, seed):
+    return np.random.default_rng(seed).standard_normal(shape)
+
+
+# ---------------------------------------------------------------------------
+# Pin functions.  Each takes the two oracle entry points it exercises so that
+# the mutation tests can run the same checks against planted mistakes.
+# ---------------------------------------------------------------------------
+
+def pin_rows_sum_to_one(probs_fn=A.probs_head, scores_fn=A.scores_head):
+    """P >= 0 and each row of P sums to 1 (definition of the row softmax)."""
+    worst = 0.0
+    for causal in (False, True):
+        q, k = _rand((37, 8), 1), _rand((37, 8), 2)
+        p, _ = probs_fn(scores_fn(q, k, 0.35, causal))
+        if np.any(p < 0):
+            return math.inf
+        worst = max(worst, float(np.max(np.abs(p.sum(axis=1) - 1.0))))
+        if causal:
+            # hidden keys (j > i) carry exactly zero weight
+            worst = max(worst, float(np.max(np.abs(np.triu(p, 1)))))
+    return worst
+
+
+def pin_constant_scores(fwd=A.forward_head):
+    """Q = 0 gives equal scores: O_i = mean of the visible V_j, LSE_i = ln(#visible)."""
+    n, d = 23, 5
+    v = _rand((n, d), 3)
+    k = _rand((n, d), 4)
+    q = np.zeros((n, d))
+    worst = 0.0
+    o, lse = fwd(q, k, v, 0.7, False)
+    worst = max(worst, np.max(np.abs(o - v.mean(axis=0))), np.max(np.abs(lse - math.log(n))))
+    o, lse = fwd(q, k, v, 0.7, True)
+    counts = np.arange(1, n + 1)
+    want = np.cumsum(v, axis=0) / counts[:, None]
+    worst = max(worst, np.max(np.abs(o - want)), np.max(np.abs(lse - np.log(counts))))
+    # all key rows equal: the score of row i is the constant c_i = scale*<q_i, k>
+    q = _rand((n, d), 5)
+    krow = _rand((1, d), 6)
+    kk = np.repeat(krow, n, axis=0)
+    o, lse = fwd(q, kk, v, 0.3, False)
+    c = 0.3 * (q @ krow[0])
+    worst = max(worst, np.max(np.abs(o - v.mean(axis=0))), np.max(np.abs(lse - (c + math.log(n)))))
+    return float(worst)
+
+
+def pin_dominant_key(fwd=A.forward_head):
+    """One key scores t, all others 0: O_i = (e^t v_* + sum_{others} v_j) / (e^t + #others)."""
+    n = d = 12
+    t = 9.0
+    k = np.eye(n, d)                      # orthonormal keys
+    v = _rand((n, d), 7)
+    star = (np.arange(n) * 5 + 3) % n     # a different target key per query
+    q = t * k[star]                       # <q_i, k_j> = t if j == star_i else 0
+    worst = 0.0
+    o, lse = fwd(q, k, v, 1.0, False)
+    for i in range(n):
+        num = math.exp(t) * v[star[i]] + (v.sum(axis=0) - v[star[i]])
+        den = math.exp(t) + (n - 1)
+        worst = max(worst, np.max(np.abs(o[i] - num / den)), abs(lse[i] - math.log(den)))
+    # causal: only keys j <= i are visible
+    star_c = np.array([(i * 7) % (i + 1) for i in range(n)])
+    q = t * k[star_c]
+    o, lse = fwd(q, k, v, 1.0, True)
+    for i in range(n):
+        vis = v[: i + 1]
+        num = math.exp(t) * v[star_c[i]] + (vis.sum(axis=0) - v[star_c[i]])
+        den = math.exp(t) + i
+        worst = max(worst, np.max(np.abs(o[i] - num / den)), abs(lse[i] - math.log(den)))
+    return float(worst)
+
+
+def pin_permutation(fwd=A.forward_head):
+    """Non-causal attention does not depend on the order of the (k_j, v_j) pairs."""
+    q, k, v = _rand((19, 6), 8), _rand((31, 6), 9), _rand((31, 4), 10)
+    perm = np.random.default_rng(11).permutation(31)
+    o1, l1 = fwd(q, k, v, 0.4, False)
+    o2, l2 = fwd(q, k[perm], v[perm], 0.4, False)
+    return float(max(np.max(np.abs(o1 - o2)), np.max(np.abs(l1 - l2))))
+
+
+def pin_blocked_equals_full(fwd=A.forward_head, blocked=A.blocked_forward_head):
+    """The pages' online-softmax recurrence equals the full softmax (exact in fp64)."""
+    worst = 0.0
+    n, d = 70, 8
+    q, k, v = _rand((n, d), 12), 3 * _rand((n, d), 13), _rand((n, d), 14)
+    for causal in (False, True):
+        o, lse = fwd(q, k, v, 0.5, causal)
+        for block in (1, 7, 16, 32, 256):
+            for tau in (0.0, 2.0, math.log(256.0)):
+                ob, lb = blocked(q, k, v, 0.5, causal, block, tau)
+                worst = max(worst, np.max(np.abs(ob - o)), np.max(np.abs(lb - lse)))
+    return float(worst)
+
+
+def pin_finite_differences(fwd=A.forward_head, bwd=A.backward_head, causal=False):
+    """Central differences of L = sum(dO * O) against (dQ, dK, dV)."""
+    n, d = 6, 3
+    q, k, v, do = (_rand((n, d), s) for s in (20, 21, 22, 23))
+    scale = 0.8
+    dq, dk, dv, _ = bwd(q, k, v, do, scale, causal)
+    h = 1e-6
+    worst = 0.0
+    for which, grad in ((0, dq), (1, dk), (2, dv)):
+        for idx in np.ndindex(n, d):
+            args = [q.copy(), k.copy(), v.copy()]
+            args[which][idx] += h
+            lp = float(np.sum(do * fwd(*args, scale, causal)[0]))
+            args[which][idx] -= 2 * h
+            lm = float(np.sum(do * fwd(*args, scale, causal)[0]))
+            fd = (lp - lm) / (2 * h)
+            worst = max(worst, abs(fd - grad[idx]) / (1.0 + abs(fd)))
+    return float(worst)
+
+
+def pin_d_identity(bwd=A.backward_head):
+    """D_i = sum_k dO_ik O_ik equals sum_j P_ij dP_ij with dP = dO V^T."""
+    n, d = 17, 4
+    q, k, v, do = (_rand((n, d), s) for s in (30, 31, 32, 33))
+    worst = 0.0
+    for causal in (False, True):
+        _, _, _, dvec = bwd(q, k, v, do, 0.6, causal)
+        p, _ = A.probs_head(A.scores_head(q, k, 0.6, causal))
+        other = np.sum(p * (do @ v.T), axis=1)
+        worst = max(worst, float(np.max(np.abs(dvec - other))))
+    return worst
+
+
+def pin_autograd(bwd=A.backward_head, fwd=A.forward_head):
+    """torch.autograd in float64 on CPU (a library routine) agrees with the oracle."""
+    worst = 0.0
+    for causal in (False, True):
+        n, d = 21, 5
+        q, k, v, do = (_rand((n, d), s) for s in (40, 41, 42, 43))
+        tq, tk, tv = (torch.tensor(x, requires_grad=True) for x in (q, k, v))
+        mask = None
+        if causal:
+            mask = torch.ones(n, n, dtype=torch.bool).tril()
+        out = torch.nn.functional.scaled_dot_product_attention(
+            tq[None, None], tk[None, None], tv[None, None], attn_mask=mask, scale=0.45)[0, 0]
+        out.backward(torch.tensor(do))
+        o, _ = fwd(q, k, v, 0.45, causal)
+        dq, dk, dv, _ = bwd(q, k, v, do, 0.45, causal)
+        worst = max(worst, float(np.max(np.abs(o - out.detach().numpy()))))
+        for a, b in ((dq, tq.grad), (dk, tk.grad), (dv, tv.grad)):
+            worst = max(worst, float(np.max(np.abs(a - b.numpy()))))
+    return worst
+
+
+# ---------------------------------------------------------------------------
+# The pins themselves
+# ---------------------------------------------------------------------------
+
+def test_rows_sum_to_one():
+    assert pin_rows_sum_to_one() < 1e-14
+
+
+def test_constant_scores_closed_form():
+    assert pin_constant_scores() < 1e-12
+
+
+def test_dominant_key_closed_form():
+    assert pin_dominant_key() < 1e-12
+
+
+def test_permutation_invariance():
+    assert pin_permutation() < 1e-13
+
+
+def test_blocked_online_softmax_equals_full():
+    assert pin_blocked_equals_full() < 1e-12
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_backward_finite_differences(causal):
+    assert pin_finite_differences(causal=causal) < 1e-7
+
+
+def test_d_identity():
+    assert pin_d_identity() < 1e-12
+
+
+def test_autograd_cross_check():
+    assert pin_autograd() < 1e-12
+
+
+def test_rows_subset_matches_definition_on_those_rows():
+    n, d = 40, 8
+    q, k, v = _rand((n, d), 50), _rand((n, d), 51), _rand((n, d), 52)
+    rows = [0, 5, 17, 39]
+    for causal in (False, True):
+        # the full-row closed form for query 0 under causal masking: only key 0
+        o_r, l_r = A.forward_rows_head(q, k, v, rows, 0.3, causal)
+        if causal:
+            assert np.max(np.abs(o_r[0] - v[0])) < 1e-15
+            assert abs(l_r[0] - 0.3 * float(q[0] @ k[0])) < 1e-14
+        o, l = A.forward_head(q, k, v, 0.3, causal)
+        assert np.max(np.abs(o_r - o[rows])) < 1e-13
+        assert np.max(np.abs(l_r - l[rows])) < 1e-13
+
+
+def test_batched_layout_maps_heads():
+    """[B, N, H, d] inputs and [B, H, N] LSE: a zero-query head reduces to mean(V)."""
+    B, N, H, d = 2, 9, 3, 4
+    g = np.random.default_rng(60)
+    Q, K, V = (g.standard_normal((B, N, H, d)) for _ in range(3))
+    Q[1, :, 2] = 0.0
+    O, LSE = oracle.forward(Q, K, V, 0.5, False)
+    assert np.max(np.abs(O[1, :, 2] - V[1, :, 2].mean(axis=0))) < 1e-13
+    assert np.max(np.abs(LSE[1, 2] - math.log(N))) < 1e-13
+    # the other heads are untouched by head (1, 2)'s inputs
+    Q2 = Q.copy()
+    Q2[1, :, 2] = 5.0
+    O2, _ = oracle.forward(Q2, K, V, 0.5, False)
+    mask = np.ones((B, H), bool)
+    mask[1, 2] = False
+    for b in range(B):
+        for h in range(H):
+            if mask[b, h]:
+                assert np.array_equal(O[b, :, h], O2[b, :, h])
+    dQ, dK, dV = oracle.backward(Q, K, V, np.ones_like(Q), 0.5, False)
+    # with dO = 1 and Q = 0 on head (1,2): dV_j = sum_i P_ij = N * (1/N) = 1
+    assert np.max(np.abs(dV[1, :, 2] - 1.0)) < 1e-13
+
+
+def test_fully_masked_row_is_zero_with_minus_inf_lse():
+    s = np.array([[-np.inf, -np.inf], [0.0, -np.inf]])
+    p, lse = A.probs_head(s)
+    assert np.all(p[0] == 0) and lse[0] == -np.inf
+    assert p[1, 0] == 1.0 and lse[1] == 0.0
+
+
+def test_pages_demo_fp32_error_magnitude():
+    """The pages' fp32 demonstration: blocked vs full differ by ~4.3e-07."""
+    g = json.loads((GOLDEN / "online_softmax_demo.json").read_text())
+    n, d, block = g["n"], g["d"], g["block"]
+    torch.manual_seed(g["seed"])
+    q, k, v = (t.numpy() for t in torch.randn(3, n, d).unbind(0))
+    scale = 1.0 / math.sqrt(d)
+    ob, _ = A.blocked_forward_head(q, k, v, np.float32(scale), False, block, 0.0, dtype=np.float32)
+    assert ob.dtype == np.float32
+    # full fp32 standard attention through torch's own softmax (library routine)
+    tq, tk, tv = (torch.from_numpy(x) for x in (q, k, v))
+    full = (torch.softmax(tq @ tk.T / math.sqrt(d), dim=-1) @ tv).numpy()
+    diff = float(np.max(np.abs(ob - full)))
+    printed = g["printed_max_abs_diff"]
+    assert printed / 10 <= diff <= printed * 10, diff
+    # in fp64 the same recurrence is exact to rounding of fp64
+    o64, _ = A.forward_head(q, k, v, scale, False)
+    ob64, _ = A.blocked_forward_head(q, k, v, scale, False, block, 0.0)
+    assert float(np.max(np.abs(ob64 - o64))) < 1e-12
+    # and both fp32 results sit within fp32 rounding of the fp64 truth
+    assert float(np.max(np.abs(full - o64))) < 10 * printed
+
+
+def test_memory_arithmetic_of_the_score_matrix():
+    """The pages' sizes for the materialised score matrix that the kernel avoids."""
+    g = json.loads((GOLDEN / "memory_arithmetic.json").read_text())
+    c = {x["what"]: x for x in g["cases"]}
+    assert 4096 ** 2 >= c["score entries at N=4096"]["entries_at_least"]
+    e8k = 8192 ** 2
+    assert abs(e8k - 67e6) / 67e6 < 0.01
+    assert abs(e8k * 2 / 2 ** 20 - 128) < 1e-9
+    assert e8k * 2 * 32 / 2 ** 30 >= 4
+    assert 256 * 256 * 2 / 1024 == 128
+    assert 16384 ** 2 * 2 / 2 ** 20 == 512
+    # the oracle really materialises N x N per head
+    s = A.scores_head(np.zeros((64, 4)), np.zeros((64, 4)), 1.0, False)
+    assert s.shape == (64, 64)
+
+
+# ---------------------------------------------------------------------------
+# Mutation tests: plausible mistakes planted in copies of the oracle.
+# ---------------------------------------------------------------------------
+
+def _mut_fwd(kind):
+    def fwd(q, k, v, scale, causal):
+        q, k, v = (np.asarray(x, float) for x in (q, k, v))
+        sc = scale
+        if kind == "no_scale":
+            sc = 1.0
+        s = sc * (q @ k.T)
+        if kind == "transposed_scores":
+            s = s.T
+        if causal:
+            hidden = np.arange(k.shape[0])[None, :] > np.arange(q.shape[0])[:, None]
+            if kind == "mask_direction":
+                hidden = hidden.T
+            if kind == "mask_diagonal":
+                hidden = np.arange(k.shape[0])[None, :] >= np.arange(q.shape[0])[:, None]
+            s = np.where(hidden, -np.inf, s)
+        m = s.max(axis=1, keepdims=True)
+        e = np.exp(s - m)
+        l = e.sum(axis=1, keepdims=True)
+        if kind == "sum_over_columns":
+            l = e.sum(axis=0, keepdims=True).T
+        p = e / l
+        lse = m[:, 0] + np.log(l[:, 0])
+        if kind == "lse_base2":
+            lse = m[:, 0] + np.log2(l[:, 0])
+        if kind == "lse_drops_max":
+            lse = np.log(l[:, 0])
+        out = p @ v
+        if kind == "values_are_keys":
+            out = p @ k[:, : v.shape[1]]
+        return out, lse
+    return fwd
+
+
+def _mut_bwd(kind):
+    def bwd(q, k, v, do, scale, causal):
+        q, k, v, do = (np.asarray(x, float) for x in (q, k, v, do))
+        p, _ = A.probs_head(A.scores_head(q, k, scale, causal))
+        o = p @ v
+        dv = p.T @ do
+        if kind == "dv_untransposed":
+            dv = p @ do
+        dp = do @ v.T
+        dvec = np.sum(do * o, axis=1)
+        ds = p * (dp - dvec[:, None])
+        if kind == "ds_sign":
+            ds = p * (dp + dvec[:, None])
+        if kind == "ds_drops_d":
+            ds = p * dp
+        dq = scale * (ds @ k)
+        dk = scale * (ds.T @ q)
+        if kind == "dk_no_scale":
+            dk = ds.T @ q
+        if kind == "dq_uses_v":
+            dq = scale * (ds @ v)
+        return dq, dk, dv, dvec
+    return bwd
+
+
+def _caught(pin, impl, tol=1e-9):
+    """A pin catches a mutant when it reports a large residual or cannot run at all."""
+    try:
+        return not (pin(impl) <= tol)
+    except (ValueError, IndexError, FloatingPointError):
+        return True
+
+
+@pytest.mark.parametrize("kind", ["no_scale", "transposed_scores", "mask_direction", "mask_diagonal",
+                                  "sum_over_columns", "lse_base2", "lse_drops_max", "values_are_keys"])
+def test_forward_mutants_are_caught(kind):
+    f = _mut_fwd(kind)
+    fails = [
+        _caught(pin_constant_scores, f),
+        _caught(pin_dominant_key, f),
+        _caught(pin_permutation, f),
+        _caught(pin_blocked_equals_full, f),
+        _caught(lambda g: pin_autograd(fwd=g), f),
+    ]
+    assert any(fails), kind
+
+
+@pytest.mark.parametrize("kind", ["dv_untransposed", "ds_sign", "ds_drops_d", "dk_no_scale", "dq_uses_v"])
+def test_backward_mutants_are_caught(kind):
+    b = _mut_bwd(kind)
+    fails = [_caught(lambda g, c=c: pin_finite_differences(bwd=g, causal=c), b) for c in (False, True)]
+    assert any(fails), kind
