@@ -1,0 +1,396 @@
+#!/usr/bin/env python
+"""Attention TFLOP/s on B200: fused forward + recomputing backward, bf16.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step is one pass of the whole hot path over one batch of synthetic input:
+the fused forward (O and LSE) followed by the backward (preprocess, main
+kernel, dQ conversion) producing dQ, dK and dV.  Workload: bf16 B=1, H=32,
+N=16384, d=128, non-causal, Q/K/V/dO i.i.d. N(0,1) with 1% of K rows scaled by
+3 (seeded; one seed per rank).  Every tensor is 128 MiB, larger than the L2,
+so no flush is needed between steps.
+
+Throughput counts 4*B*H*N^2*d FLOPs for the forward and 2.5x that for the
+backward; `value` = all ranks' FLOPs / the slowest rank's device time for K
+steps (CUDA events on the launching stream, barrier + synchronize on both
+sides).  With --gpus N > 1 (launched by torchrun) each rank runs its own copy
+of the workload: the problem shards into independent (b, h) heads, so there is
+no collective on the data path (weak scaling).
+
+--impl reference times the CPU oracle (fp64, materialises S and P) on the
+host cores: each step is one (b, h) head of the same workload, forward and
+backward; rank 0 alone runs it.
+
+Prints one JSON line.
+"""
+
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import pathlib
+import re
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = pathlib.Path(__file__).resolve().parent
+sys.path.insert(0, str(ROOT))
+
+METRIC = "attention TFLOP/s (fwd, fwd+bwd) bf16 on 1 B200 and % of dense BF16 tensor peak"
+WORKLOAD = dict(B=1, H=32, N=16384, d=128, causal=False, spike_frac=0.01, spike=3.0)
+WORKLOAD_NAME = "bf16 fwd+bwd B1 H32 N16384 d128 non-causal, K rows x3 at 1% of positions"
+FALLBACK_PEAK_TFLOPS = 1590.0  # earlier burst measurement of cuBLAS bf16 on this machine
+
+
+def flops_fwd(B, H, N, d, causal):
+    f = 4.0 * B * H * N * N * d
+    return f / 2 if causal else f
+
+
+def read_peaks():
+    p = ROOT / "MEASURED_PEAKS.json"
+    if p.exists():
+        j = json.loads(p.read_text())
+        return float(j["bf16_tflops"]), float(j.get("bf16_tflops_sustained", j["bf16_tflops"])), "measured"
+    return FALLBACK_PEAK_TFLOPS, 1400.0, "fallback"
+
+
+def read_profile_traffic(kernel_key: str):
+    """DRAM bytes per launch from the committed ncu summary, if it matches the current source."""
+    prof = ROOT / "profiles" / f"{kernel_key}.md"
+    if not prof.exists():
+        return None
+    text = prof.read_text()
+    m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    h = re.search(r"source_sha256:\s*([0-9a-f]+)", text)
+    if not m or not h:
+        return None
+    import hashlib
+    src = {"fwd_bf16": "fa_fwd_bf16.cu", "bwd_main": "fa_bwd.cu"}[kernel_key]
+    cur = hashlib.sha256((ROOT / "exact_io_aware_51_b200" / "csrc" / src).read_bytes()).hexdigest()
+    return float(m.group(1)) if cur.startswith(h.group(1)) else None
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons while the GPU is busy."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.5)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        for line in pathlib.Path(self.path).read_text().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), float(parts[3]), parts[5:9]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        loaded = [r for r in rows if r[2] > 250.0] or rows
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        reasons = sorted({names[i] for r in loaded for i, v in enumerate(r[3]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in loaded), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(loaded)}
+
+
+def cpu_cores():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads") for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n and n[0]:
+            return int(n[0])
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+def oracle_head_step(q, k, v, do, scale, causal):
+    """Time the CPU oracle on one (b, h) head: forward then backward."""
+    import oracle
+    t0 = time.perf_counter()
+    oracle.forward_head(q, k, v, scale, causal)
+    oracle.backward_head(q, k, v, do, scale, causal)
+    return time.perf_counter() - t0
+
+
+def head_inputs(seed=0):
+    import numpy as np
+    from exact_io_aware_51_b200 import inputs as I
+    w = WORKLOAD
+    q, k, v, do = I.make_inputs(w["B"], w["N"], w["H"], w["d"], seed=seed, spike_frac=w["spike_frac"],
+                                spike=w["spike"])
+    return tuple(t[0, :, 0].float().numpy().astype(np.float64) for t in (q, k, v, do))
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1 and args.impl == "ours":
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return None
+    w = WORKLOAD
+    scale = float(1.0 / math.sqrt(w["d"]))
+    q, k, v, do = head_inputs(0)
+    for _ in range(args.warmup):
+        oracle_head_step(q, k, v, do, scale, w["causal"])
+    times = [oracle_head_step(q, k, v, do, scale, w["causal"]) for _ in range(args.steps)]
+    f_head = flops_fwd(1, 1, w["N"], w["d"], w["causal"])
+    tot = sum(times)
+    value = 3.5 * f_head * args.steps / tot / 1e12
+    cores = cpu_cores()
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD_NAME, **w, "sample": "one (b, h) head per step"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": "forward + backward of one (b, h) head (N=16384, d=128) per step"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def run_ours(args, world, rank, local):
+    import torch
+
+    import exact_io_aware_51_b200 as fa
+    from exact_io_aware_51_b200 import inputs as I
+
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    w = WORKLOAD
+    B, H, N, d, causal = w["B"], w["H"], w["N"], w["d"], w["causal"]
+    scale = float(1.0 / math.sqrt(d))
+    q_h, k_h, v_h, do_h = I.make_inputs(B, N, H, d, seed=rank, spike_frac=w["spike_frac"], spike=w["spike"])
+    q, k, v, do = (t.to(dev) for t in (q_h, k_h, v_h, do_h))
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(fa.bwd_workspace_size(B, H, N, d), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        fa.fwd(q, k, v, causal=causal, scale=scale, out=o, lse=lse)
+        fa.bwd(q, k, v, o, do, lse, causal=causal, scale=scale, workspace=ws, dq=dq, dk=dk, dv=dv)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if dist is None:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    # ---- timed region: K steps, kernel events around the two tensor-core kernels ----
+    ev_f = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    ev_b = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    t0.record(stream)
+    for i in range(args.steps):
+        fa.set_kernel_events(*ev_f[i])
+        fa.fwd(q, k, v, causal=causal, scale=scale, out=o, lse=lse)
+        fa.set_kernel_events(*ev_b[i])
+        fa.bwd(q, k, v, o, do, lse, causal=causal, scale=scale, workspace=ws, dq=dq, dk=dk, dv=dv)
+    fa.set_kernel_events(None, None)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clocks = sampler.stop()
+    rc, detail = fa.last_device_status()
+    if rc != 0:
+        raise RuntimeError(f"device status {rc} ({detail:#x}) after the timed region")
+    ms_local = t0.elapsed_time(t1)
+    ms = max_over_ranks(ms_local)
+    fwd_ms = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in ev_f))
+    bwd_main_ms = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in ev_b))
+
+    f = flops_fwd(B, H, N, d, causal)
+    total_flops = 3.5 * f * args.steps * world
+    value = total_flops / (ms * 1e-3) / 1e12
+    ms_step = ms / args.steps
+    peak_burst, peak_sustained, peak_src = read_peaks()
+    fwd_tflops = f / (fwd_ms * 1e-3) / 1e12
+    bwd_main_tflops = 2.5 * f / (bwd_main_ms * 1e-3) / 1e12
+    bwd_total_ms = ms_step - fwd_ms  # preprocess + main + dQ convert
+
+    # dominant kernel of the step
+    if bwd_main_ms >= fwd_ms:
+        dom = {"kernel": "bwd_main_kernel", "flops": 2.5 * f, "ms": bwd_main_ms, "key": "bwd_main"}
+    else:
+        dom = {"kernel": "fwd_bf16_kernel", "flops": f, "ms": fwd_ms, "key": "fwd_bf16"}
+    achieved = dom["flops"] / (dom["ms"] * 1e-3) / 1e12
+    roofline = {"bound": "tensor", "kernel": dom["kernel"], "achieved": achieved, "peak": peak_burst,
+                "peak_source": f"{peak_src} bf16 burst (cuBLAS)", "unit": "TFLOP/s", "frac": achieved / peak_burst,
+                "traffic": read_profile_traffic(dom["key"]),
+                "flops_per_launch": dom["flops"], "ms_per_launch": dom["ms"]}
+
+    # ---- end to end through the public API with host buffers ----
+    pin = [t.pin_memory() for t in (q_h, k_h, v_h, do_h)]
+    out_h = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (o, lse, dq, dk, dv)]
+    h2d = sum(t.numel() * t.element_size() for t in pin)
+    d2h = sum(t.numel() * t.element_size() for t in out_h)
+    e_steps = max(1, min(args.steps, 10))
+
+    def e2e_step():
+        for dst, src in zip((q, k, v, do), pin):
+            dst.copy_(src, non_blocking=True)
+        step()
+        for dst, src in zip(out_h, (o, lse, dq, dk, dv)):
+            dst.copy_(src, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1))
+    e2e_value = 3.5 * f * e_steps * world / (e2e_ms * 1e-3) / 1e12
+
+    result = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": WORKLOAD_NAME, "B": B, "H": H, "N": N, "d": d, "causal": causal,
+                   "global_batch": B * world, "seq_len": N,
+                   "parallelism": f"replicas: one independent workload per GPU ({world})",
+                   "l2": "inputs larger than L2 (each of Q, K, V, O, dO is 128 MiB); no flush"},
+        "fwd": {"tflops": fwd_tflops, "frac_of_peak": fwd_tflops / peak_burst, "ms": fwd_ms},
+        "bwd": {"tflops": 2.5 * f / (bwd_total_ms * 1e-3) / 1e12, "ms": bwd_total_ms,
+                "main_kernel_tflops": bwd_main_tflops, "main_kernel_ms": bwd_main_ms,
+                "main_frac_of_peak": bwd_main_tflops / peak_burst},
+        "frac_of_peak": value / world / peak_burst,
+        "peak_tflops": {"burst": peak_burst, "sustained": peak_sustained, "source": peak_src},
+        "roofline": roofline,
+        "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "steps": e_steps},
+        "gpu_launches": 4 * args.steps,
+        "clocks": clocks,
+    }
+    del pin, out_h
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        qh, kh, vh, doh = (t[0, :, 0].float().numpy().astype("float64") for t in (q_h, k_h, v_h, do_h))
+        t = oracle_head_step(qh, kh, vh, doh, scale, causal)
+        result["cpu_baseline"] = {
+            "value": 3.5 * flops_fwd(1, 1, N, d, causal) / t / 1e12, "unit": "TFLOP/s", "cores": cpu_cores(),
+            "kind": "oracle", "sample": "forward + backward of one (b, h) head (N=16384, d=128), fp64",
+            "seconds": t}
+    return result
+
+
+PROFILE_WORKLOAD = dict(B=1, H=64, N=4096, d=128)
+
+
+def run_profile_case(args):
+    """Small case for ncu section captures: 2 x (forward, backward) on B1 H64 N4096 d128
+    (each tensor 64 MiB, so the five of them exceed the L2; < 1 GB on the device)."""
+    import torch
+
+    import exact_io_aware_51_b200 as fa
+    from exact_io_aware_51_b200 import inputs as I
+    w = PROFILE_WORKLOAD
+    q, k, v, do = (t.cuda() for t in I.make_inputs(w["B"], w["N"], w["H"], w["d"], seed=0))
+    for causal in ((False, True) if args.profile_causal else (False,)):
+        for _ in range(2):
+            o, lse = fa.fwd(q, k, v, causal=causal)
+            fa.bwd(q, k, v, o, do, lse, causal=causal)
+    torch.cuda.synchronize()
+    rc, detail = fa.last_device_status()
+    if rc != 0:
+        raise RuntimeError(f"device status {rc} ({detail:#x})")
+    print(json.dumps({"profile_case": w, "ok": True}))
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing on the host")
+    ap.add_argument("--profile-case", action="store_true",
+                    help="run only the small profiling case (2 x fwd + bwd, B1 H64 N4096 d128) for ncu")
+    ap.add_argument("--profile-causal", action="store_true", help="with --profile-case: also the causal pair")
+    args = ap.parse_args()
+    if args.profile_case:
+        run_profile_case(args)
+        return
+    if args.warmup < 3 and args.impl == "ours":
+        ap.error("--warmup must be >= 3")
+    world, rank, local = dist_setup(args)
+    try:
+        if args.impl == "reference":
+            res = run_reference(args, world, rank)
+        else:
+            res = run_ours(args, world, rank, local)
+        if rank == 0 and res is not None:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1 and args.impl == "ours":
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,214 @@
+"""Exact IO-aware attention for B200 (sm_100a): Python binding of ``libfa.so``.
+
+This module only marshals arguments: it checks tensor shapes, dtypes and
+devices, allocates outputs with PyTorch (PyTorch is used for device memory and
+streams only), and calls the C ABI declared in ``include/fa.h`` through
+ctypes.  Every step of the computation runs in the library's CUDA kernels;
+there is no CPU fallback.  If the library is missing, every call raises.
+
+    o, lse = fwd(q, k, v, causal=False)          # q, k, v: [B, N, H, d] cuda
+    dq, dk, dv = bwd(q, k, v, o, do, lse, causal=False)
+"""
+
+from __future__ import annotations
+
+import ctypes
+import math
+import pathlib
+
+import torch
+
+__all__ = [
+    "FAError", "FA_BF16", "FA_FP32", "lib", "lib_path", "fwd", "bwd", "bwd_workspace_size",
+    "last_device_status", "set_wait_limit_ms", "debug_inject", "debug_umma", "status_string",
+    "set_kernel_events",
+    "attention", "EXPORTED",
+]
+
+FA_BF16 = 0
+FA_FP32 = 1
+_PKG = pathlib.Path(__file__).resolve().parent
+_LIB = None
+
+# Every symbol include/fa.h declares.
+EXPORTED = ("fa_fwd", "fa_bwd_workspace_size", "fa_bwd", "fa_status_string", "fa_last_cuda_error",
+            "fa_last_device_status", "fa_set_wait_limit_ms", "fa_debug_inject", "fa_debug_umma",
+            "fa_version", "fa_set_kernel_events")
+
+
+class FAError(RuntimeError):
+    """A non-zero status from the C library (``status`` holds the code)."""
+
+    def __init__(self, status: int, what: str = ""):
+        self.status = int(status)
+        msg = status_string(status) if _LIB is not None else f"status {status}"
+        if self.status == -6 and _LIB is not None:
+            msg += f" (cudaError {_LIB.fa_last_cuda_error()})"
+        super().__init__(f"{what}: {msg}" if what else msg)
+
+
+def lib_path() -> pathlib.Path:
+    return _PKG / "libfa.so"
+
+
+def lib() -> ctypes.CDLL:
+    """Load ``libfa.so`` (built by ``python -m exact_io_aware_51_b200.build``)."""
+    global _LIB
+    if _LIB is not None:
+        return _LIB
+    path = lib_path()
+    if not path.exists():
+        raise FAError(-6, f"{path} is missing; build it with `python -m exact_io_aware_51_b200.build`")
+    L = ctypes.CDLL(str(path))
+    vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    L.fa_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, i, vp]
+    L.fa_fwd.restype = i
+    L.fa_bwd_workspace_size.argtypes = [i, i, i, i, i]
+    L.fa_bwd_workspace_size.restype = sz
+    L.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, i, vp, sz, vp]
+    L.fa_bwd.restype = i
+    L.fa_status_string.argtypes = [i]
+    L.fa_status_string.restype = ctypes.c_char_p
+    L.fa_last_cuda_error.argtypes = []
+    L.fa_last_cuda_error.restype = i
+    L.fa_last_device_status.argtypes = [vp, ctypes.POINTER(i)]
+    L.fa_last_device_status.restype = i
+    L.fa_set_wait_limit_ms.argtypes = [i]
+    L.fa_set_wait_limit_ms.restype = None
+    L.fa_debug_inject.argtypes = [i]
+    L.fa_debug_inject.restype = None
+    L.fa_debug_umma.argtypes = [vp, vp, vp, i, i, i, i, i, vp]
+    L.fa_debug_umma.restype = i
+    L.fa_set_kernel_events.argtypes = [vp, vp]
+    L.fa_set_kernel_events.restype = None
+    L.fa_version.argtypes = []
+    L.fa_version.restype = i
+    _LIB = L
+    return L
+
+
+def status_string(status: int) -> str:
+    return lib().fa_status_string(int(status)).decode()
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return FA_BF16
+    if t.dtype == torch.float32:
+        return FA_FP32
+    raise TypeError(f"unsupported dtype {t.dtype}; use bfloat16 or float32")
+
+
+def _stream_handle(stream, device) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    return s.cuda_stream
+
+
+def _check_inputs(*ts: torch.Tensor):
+    t0 = ts[0]
+    if t0.dim() != 4:
+        raise ValueError("expected [B, N, H, d] tensors")
+    if not t0.is_cuda:
+        raise ValueError("tensors must live on a CUDA device (there is no CPU path)")
+    for t in ts:
+        if t.shape != t0.shape or t.dtype != t0.dtype or t.device != t0.device:
+            raise ValueError("q, k, v (and o, do) must share shape, dtype and device")
+        if not t.is_contiguous():
+            raise ValueError("tensors must be contiguous [B, N, H, d]")
+
+
+def _scale(scale, d):
+    return float(1.0 / math.sqrt(d)) if scale is None else float(scale)
+
+
+def fwd(q, k, v, causal: bool = False, scale: float | None = None, out=None, lse=None, stream=None):
+    """Forward pass: returns (o [B, N, H, d], lse [B, H, N] fp32)."""
+    _check_inputs(q, k, v)
+    B, N, H, d = q.shape
+    o = torch.empty_like(q) if out is None else out
+    l = torch.empty((B, H, N), dtype=torch.float32, device=q.device) if lse is None else lse
+    rc = lib().fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), l.data_ptr(), B, H, N, d,
+                      _scale(scale, d), int(bool(causal)), _dtype_code(q), _stream_handle(stream, q.device))
+    if rc != 0:
+        raise FAError(rc, "fa_fwd")
+    return o, l
+
+
+def bwd_workspace_size(B: int, H: int, N: int, d: int, dtype: int = FA_BF16) -> int:
+    return int(lib().fa_bwd_workspace_size(B, H, N, d, dtype))
+
+
+def bwd(q, k, v, o, do, lse, causal: bool = False, scale: float | None = None, workspace=None,
+        dq=None, dk=None, dv=None, stream=None):
+    """Backward pass by recomputation: returns (dq, dk, dv), each [B, N, H, d]."""
+    _check_inputs(q, k, v, o, do)
+    B, N, H, d = q.shape
+    if lse.shape != (B, H, N) or lse.dtype != torch.float32 or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous fp32 [B, H, N] tensor")
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    need = bwd_workspace_size(B, H, N, d, _dtype_code(q))
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    rc = lib().fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(), lse.data_ptr(),
+                      dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, N, d, _scale(scale, d),
+                      int(bool(causal)), _dtype_code(q), workspace.data_ptr(), workspace.numel(),
+                      _stream_handle(stream, q.device))
+    if rc != 0:
+        raise FAError(rc, "fa_bwd")
+    return dq, dk, dv
+
+
+def last_device_status(stream=None, device=None):
+    """Synchronise and read/clear the device status word: (status, raw word)."""
+    detail = ctypes.c_int(0)
+    dev = device if device is not None else torch.cuda.current_device()
+    rc = lib().fa_last_device_status(_stream_handle(stream, dev), ctypes.byref(detail))
+    return rc, detail.value
+
+
+def set_wait_limit_ms(ms: int):
+    lib().fa_set_wait_limit_ms(int(ms))
+
+
+def debug_inject(mode: int):
+    lib().fa_debug_inject(int(mode))
+
+
+def set_kernel_events(start=None, stop=None):
+    """Record torch.cuda.Event pairs around the next calls' tensor-core kernel (None, None: off)."""
+    lib().fa_set_kernel_events(start.cuda_event if start is not None else None,
+                               stop.cuda_event if stop is not None else None)
+
+
+def debug_umma(a: torch.Tensor, b: torch.Tensor, a_mn_major: int, b_mn_major: int, a_tmem: int = 0,
+               stream=None) -> torch.Tensor:
+    """One tcgen05 MMA tile D = A B^T (test-only): a [128, K], b [N, K] bf16 cuda."""
+    n, kdim = b.shape
+    dmat = torch.empty((128, n), dtype=torch.float32, device=a.device)
+    rc = lib().fa_debug_umma(a.data_ptr(), b.data_ptr(), dmat.data_ptr(), n, kdim, int(a_mn_major),
+                             int(b_mn_major), int(a_tmem), _stream_handle(stream, a.device))
+    if rc != 0:
+        raise FAError(rc, "fa_debug_umma")
+    return dmat
+
+
+class _Attention(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, q, k, v, causal, scale):
+        o, lse = fwd(q, k, v, causal=causal, scale=scale)
+        ctx.save_for_backward(q, k, v, o, lse)
+        ctx.causal, ctx.scale = causal, scale
+        return o
+
+    @staticmethod
+    def backward(ctx, do):
+        q, k, v, o, lse = ctx.saved_tensors
+        dq, dk, dv = bwd(q, k, v, o, do.contiguous(), lse, causal=ctx.causal, scale=ctx.scale)
+        return dq, dk, dv, None, None
+
+
+def attention(q, k, v, causal: bool = False, scale: float | None = None):
+    """Differentiable attention over [B, N, H, d] tensors (forward + recomputing backward)."""
+    return _Attention.apply(q, k, v, causal, scale)

@@ -1,0 +1,331 @@
+// Host side of the C ABI: argument validation, TMA descriptors, per-device
+// state and kernel launches.  See include/fa.h for the contract.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstdlib>
+#include <mutex>
+
+#include "fa.h"
+#include "fa_internal.h"
+
+namespace fa {
+
+// Device status word and the epoch of the last launch that hit a wait limit.
+__device__ int g_status;
+__device__ unsigned int g_abort_epoch;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr long long kMaxN = 1LL << 22;
+
+thread_local int t_last_cuda_error = 0;
+thread_local cudaEvent_t t_ev_start = nullptr;
+thread_local cudaEvent_t t_ev_stop = nullptr;
+std::atomic<unsigned int> g_epoch{1};
+std::atomic<unsigned long long> g_limit_ns{0};
+std::atomic<int> g_inject{0};
+
+struct DeviceState {
+  std::once_flag once;
+  int arch_ok = 0;
+  int init_err = 0;
+  int* status = nullptr;
+  unsigned int* abort_epoch = nullptr;
+};
+DeviceState g_dev[kMaxDevices];
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+unsigned long long wait_limit_ns() {
+  unsigned long long v = g_limit_ns.load();
+  if (v == 0) {
+    const char* e = std::getenv("FA_TIMEOUT_MS");
+    long long ms = e ? std::atoll(e) : 2000;
+    if (ms <= 0) ms = 2000;
+    v = static_cast<unsigned long long>(ms) * 1000000ull;
+    g_limit_ns.store(v);
+  }
+  return v;
+}
+
+int fail_cuda(cudaError_t e) {
+  t_last_cuda_error = static_cast<int>(e);
+  return FA_ERR_LAUNCH;
+}
+
+// A failed TMA descriptor encode is reported as 100000 + the CUresult.
+int fail_encode(CUresult r) {
+  t_last_cuda_error = 100000 + static_cast<int>(r);
+  return FA_ERR_LAUNCH;
+}
+
+// Per-device one-time set-up: architecture check and the device addresses of
+// the status word and abort epoch (done with that device current).
+int device_state(DeviceState** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail_cuda(e);
+  if (dev < 0 || dev >= kMaxDevices) return FA_ERR_ARCH;
+  DeviceState& st = g_dev[dev];
+  std::call_once(st.once, [&] {
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
+      st.init_err = FA_ERR_ARCH;
+      return;
+    }
+    st.arch_ok = (major == 10 && minor == 0);
+    void* p = nullptr;
+    cudaError_t e1 = cudaGetSymbolAddress(&p, g_status);
+    if (e1 != cudaSuccess) {
+      st.init_err = fail_cuda(e1);
+      return;
+    }
+    st.status = static_cast<int*>(p);
+    cudaError_t e2 = cudaGetSymbolAddress(&p, g_abort_epoch);
+    if (e2 != cudaSuccess) {
+      st.init_err = fail_cuda(e2);
+      return;
+    }
+    st.abort_epoch = static_cast<unsigned int*>(p);
+  });
+  if (st.init_err) return st.init_err;
+  if (!st.arch_ok) return FA_ERR_ARCH;
+  *out = &st;
+  return FA_OK;
+}
+
+DevCtl make_ctl(const DeviceState& st) {
+  DevCtl c;
+  c.status = st.status;
+  c.abort_epoch = st.abort_epoch;
+  unsigned int ep = g_epoch.fetch_add(1);
+  if (ep == 0) ep = g_epoch.fetch_add(1);  // 0 never names a launch
+  c.epoch = ep;
+  c.limit_ns = wait_limit_ns();
+  c.inject = g_inject.load();
+  return c;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+int check_shape(int B, int H, int N, int d, int dtype) {
+  if (B < 0 || H < 0 || N < 0) return FA_ERR_INVALID_ARG;
+  if (dtype != FA_BF16 && dtype != FA_FP32) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (N > kMaxN || H > 65535 || B > 65535) return FA_ERR_TOO_LARGE;
+  const double elems = static_cast<double>(B) * N * H * d;
+  if (elems >= 1099511627776.0) return FA_ERR_TOO_LARGE;  // 2^40
+  return FA_OK;
+}
+
+int check_scale(float scale) {
+  if (!std::isfinite(scale) || !(scale > 0.f)) return FA_ERR_INVALID_ARG;
+  return FA_OK;
+}
+
+}  // namespace
+
+CUresult make_tile_map(CUtensorMap* map, const void* base, int B, int N, int H, int d, int rows) {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  if (!g_encode) return CUDA_ERROR_NOT_FOUND;
+  // dims innermost first: feature, sequence, head, batch
+  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(H),
+                              static_cast<cuuint64_t>(B)};
+  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(H) * d * 2, static_cast<cuuint64_t>(d) * 2,
+                                 static_cast<cuuint64_t>(N) * H * d * 2};
+  const cuuint32_t box[4] = {64u, static_cast<cuuint32_t>(rows), 1u, 1u};
+  const cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+  return g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+}
+
+}  // namespace fa
+
+using namespace fa;
+
+extern "C" {
+
+int fa_version(void) { return 100; }
+
+const char* fa_status_string(int status) {
+  switch (status) {
+    case FA_OK: return "ok";
+    case FA_ERR_INVALID_ARG: return "invalid argument (null pointer, negative size, bad scale or dtype)";
+    case FA_ERR_UNSUPPORTED: return "unsupported configuration (head dim, dtype or pass)";
+    case FA_ERR_MISALIGNED: return "tensor pointer not 16-byte aligned";
+    case FA_ERR_WORKSPACE: return "backward workspace missing, too small or misaligned";
+    case FA_ERR_ARCH: return "current CUDA device is not an sm_100 (B200-class) GPU";
+    case FA_ERR_LAUNCH: return "CUDA call failed (see fa_last_cuda_error)";
+    case FA_ERR_DEVICE_TIMEOUT: return "a kernel wait exceeded its limit; outputs of that launch are undefined";
+    case FA_ERR_TOO_LARGE: return "problem exceeds a size limit";
+    default: return "unknown status";
+  }
+}
+
+int fa_last_cuda_error(void) { return t_last_cuda_error; }
+
+void fa_set_wait_limit_ms(int ms) {
+  g_limit_ns.store(ms > 0 ? static_cast<unsigned long long>(ms) * 1000000ull : 0ull);
+}
+
+void fa_debug_inject(int mode) { g_inject.store(mode); }
+
+void fa_set_kernel_events(void* start, void* stop) {
+  t_ev_start = static_cast<cudaEvent_t>(start);
+  t_ev_stop = static_cast<cudaEvent_t>(stop);
+}
+
+int fa_last_device_status(void* stream, int* detail) {
+  DeviceState* st = nullptr;
+  int rc = device_state(&st);
+  if (rc) return rc;
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail_cuda(e);
+  int v = 0;
+  e = cudaMemcpy(&v, st->status, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return fail_cuda(e);
+  const int zero = 0;
+  e = cudaMemcpy(st->status, &zero, sizeof(int), cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) return fail_cuda(e);
+  if (detail) *detail = v;
+  return v ? FA_ERR_DEVICE_TIMEOUT : FA_OK;
+}
+
+int fa_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, int B, int H, int N, int d, float scale,
+           int causal, int dtype, void* stream) {
+  int rc = check_shape(B, H, N, d, dtype);
+  if (rc) return rc;
+  if ((rc = check_scale(scale))) return rc;
+  if (static_cast<long long>(B) * H * N == 0) return FA_OK;
+  if (!Q || !K || !V || !O || !LSE) return FA_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(LSE)) return FA_ERR_MISALIGNED;
+  DeviceState* st = nullptr;
+  if ((rc = device_state(&st))) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+  FwdArgs a;
+  a.B = B;
+  a.H = H;
+  a.N = N;
+  a.d = d;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.causal = causal ? 1 : 0;
+  a.O = O;
+  a.LSE = LSE;
+  cudaError_t e;
+  if (dtype == FA_FP32) {
+    e = launch_fwd_f32(static_cast<const float*>(Q), static_cast<const float*>(K), static_cast<const float*>(V), a, s);
+  } else {
+    CUtensorMap tq, tk, tv;
+    CUresult r;
+    if ((r = make_tile_map(&tq, Q, B, N, H, d, 128)) != CUDA_SUCCESS ||
+        (r = make_tile_map(&tk, K, B, N, H, d, 128)) != CUDA_SUCCESS ||
+        (r = make_tile_map(&tv, V, B, N, H, d, 128)) != CUDA_SUCCESS)
+      return fail_encode(r);
+    if (t_ev_start) cudaEventRecord(t_ev_start, s);
+    e = launch_fwd_bf16(tq, tk, tv, a, make_ctl(*st), s);
+    if (t_ev_stop && e == cudaSuccess) cudaEventRecord(t_ev_stop, s);
+  }
+  if (e != cudaSuccess) return fail_cuda(e);
+  return FA_OK;
+}
+
+size_t fa_bwd_workspace_size(int B, int H, int N, int d, int dtype) {
+  if (check_shape(B, H, N, d, dtype) != FA_OK) return 0;
+  if (static_cast<long long>(B) * H * N == 0) return 0;
+  const size_t npad = (static_cast<size_t>(N) + 127) / 128 * 128;
+  const size_t dq = align256(static_cast<size_t>(B) * N * H * d * sizeof(float));
+  const size_t rows = align256(static_cast<size_t>(B) * H * npad * sizeof(float));
+  return dq + 2 * rows;
+}
+
+int fa_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO, const float* LSE, void* dQ,
+           void* dK, void* dV, int B, int H, int N, int d, float scale, int causal, int dtype, void* workspace,
+           size_t workspace_bytes, void* stream) {
+  int rc = check_shape(B, H, N, d, dtype);
+  if (rc) return rc;
+  if ((rc = check_scale(scale))) return rc;
+  if (dtype != FA_BF16 || d != 128) return FA_ERR_UNSUPPORTED;
+  if (static_cast<long long>(B) * H * N == 0) return FA_OK;
+  if (!Q || !K || !V || !O || !dO || !LSE || !dQ || !dK || !dV) return FA_ERR_INVALID_ARG;
+  const void* ptrs[] = {Q, K, V, O, dO, LSE, dQ, dK, dV};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return FA_ERR_MISALIGNED;
+  const size_t need = fa_bwd_workspace_size(B, H, N, d, dtype);
+  if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return FA_ERR_WORKSPACE;
+  DeviceState* st = nullptr;
+  if ((rc = device_state(&st))) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+  const int npad = (N + 127) / 128 * 128;
+  BwdArgs a;
+  a.B = B;
+  a.H = H;
+  a.N = N;
+  a.d = d;
+  a.Npad = npad;
+  a.scale = scale;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.causal = causal ? 1 : 0;
+  a.O = O;
+  a.dO = dO;
+  a.LSE = LSE;
+  a.dQ = dQ;
+  a.dK = dK;
+  a.dV = dV;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  a.dQacc = reinterpret_cast<float*>(ws);
+  ws += align256(static_cast<size_t>(B) * N * H * d * sizeof(float));
+  a.Dvec = reinterpret_cast<float*>(ws);
+  ws += align256(static_cast<size_t>(B) * H * npad * sizeof(float));
+  a.LSE2 = reinterpret_cast<float*>(ws);
+
+  CUtensorMap tq, tk, tv, tdo;
+  CUresult r;
+  if ((r = make_tile_map(&tq, Q, B, N, H, d, 64)) != CUDA_SUCCESS ||
+      (r = make_tile_map(&tdo, dO, B, N, H, d, 64)) != CUDA_SUCCESS ||
+      (r = make_tile_map(&tk, K, B, N, H, d, 128)) != CUDA_SUCCESS ||
+      (r = make_tile_map(&tv, V, B, N, H, d, 128)) != CUDA_SUCCESS)
+    return fail_encode(r);
+  cudaError_t e = launch_bwd_pre(a, s);
+  if (e != cudaSuccess) return fail_cuda(e);
+  if (t_ev_start) cudaEventRecord(t_ev_start, s);
+  e = launch_bwd_main(tq, tk, tv, tdo, a, make_ctl(*st), s);
+  if (e != cudaSuccess) return fail_cuda(e);
+  if (t_ev_stop) cudaEventRecord(t_ev_stop, s);
+  e = launch_bwd_dq(a, s);
+  if (e != cudaSuccess) return fail_cuda(e);
+  return FA_OK;
+}
+
+int fa_debug_umma(const void* A, const void* B, float* D, int N, int K, int a_mn_major, int b_mn_major, int a_tmem,
+                  void* stream) {
+  if (!A || !B || !D) return FA_ERR_INVALID_ARG;
+  if ((N != 64 && N != 128) || (K != 64 && K != 128)) return FA_ERR_UNSUPPORTED;
+  DeviceState* st = nullptr;
+  int rc = device_state(&st);
+  if (rc) return rc;
+  cudaError_t e = launch_umma_probe(A, B, D, N, K, a_mn_major ? 1 : 0, b_mn_major ? 1 : 0, a_tmem ? 1 : 0,
+                                    static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail_cuda(e);
+  return FA_OK;
+}
+
+}  // extern "C"

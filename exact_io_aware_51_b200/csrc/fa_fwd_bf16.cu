@@ -1,0 +1,367 @@
+// Fused attention forward, bf16 inputs, fp32 accumulation, sm_100a.
+//
+// Method: "Flash Attention" (Ultralytics glossary), "Принцип работы Flash
+// Attention" -- a block of queries stays on chip while key/value blocks stream
+// past; per block the scores are formed, the running row maximum and sum are
+// updated, the partial output is rescaled when the maximum grows, and the
+// block's weighted values are added; only the output and one number per row
+// (here the log-sum-exp) go back to HBM.  "Flash Attention" (karlkratz.de),
+// "Tiling: Blockweise Berechnung im schnellen Speicher" gives the same per-row
+// maximum / sum pair and the correction factor.
+//
+// B200 design (ours; the pages' A100/H100 tilings are prior art only):
+//   * one CTA owns two 128-row query tiles (t = 0, 1) of one (b, h) and
+//     streams 128-key K/V tiles through a TMA ring in shared memory
+//     (128-byte swizzle, mbarrier completion);
+//   * one thread issues all tcgen05 MMAs: S_t = Q_t K^T (both operands from
+//     shared memory, accumulator in TMEM) and O_t += P_t V (P_t read straight
+//     from TMEM where the softmax wrote it over S_t, V from shared memory);
+//   * eight softmax warps (one TMEM lane = one query row per thread) read S_t,
+//     mask, take the row max, form P = 2^(S*scale*log2e - m) with the scale
+//     folded into one FFMA, add the row sum, and write P back as bf16;
+//   * lazy rescale: the reference maximum m only moves when a row's maximum
+//     grows by more than 2^8; numerator and denominator share m, so the result
+//     is exact and the O rescale (a TMEM read-modify-write) is rare;
+//   * causal: key tiles beyond the query tile's diagonal are never visited and
+//     only the diagonal tile is masked; CTAs with longer rows start first;
+//   * epilogue: O / l -> bf16 with 16-byte stores, LSE = (m + log2 l) ln 2.
+// The two query tiles ping-pong: while the softmax of one tile runs, the
+// tensor pipe computes the other tile's products.
+#include <cuda_bf16.h>
+
+#include "fa_internal.h"
+#include "sm100.cuh"
+
+namespace fa {
+namespace {
+
+constexpr int kBM = 128;        // query rows per tile = TMEM lanes
+constexpr int kBN = 128;        // keys per K/V tile
+constexpr int kThreads = 384;   // WG0, WG1: softmax; WG2: loader warp, MMA warp, 2 spare
+// Register split (per thread): 384 x 168 at launch = 256 x 216 + 128 x 72.
+constexpr uint32_t kRegSoftmax = 216;
+constexpr uint32_t kRegOther = 72;
+constexpr float kTau = 8.0f;    // lazy-rescale threshold (log2 units)
+
+template <int D>
+struct FwdCfg {
+  static constexpr int kSub = D / 64;                 // 64-feature sub-tiles per row
+  static constexpr int kSubBytes = kBM * 128;         // one [128][64] bf16 sub-tile
+  static constexpr int kTileBytes = kSub * kSubBytes; // one 128 x D tile
+  static constexpr int kStages = (D == 128) ? 2 : 4;
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffK = 2 * kTileBytes;
+  static constexpr int kOffV = kOffK + kStages * kTileBytes;
+  static constexpr int kOffBar = kOffV + kStages * kTileBytes;
+  static constexpr int kSmemBytes = kOffBar + 512 + 1024;  // barriers + base alignment slack
+  // TMEM columns: S_0 | S_1 | O_0 | O_1
+  __device__ static constexpr uint32_t colS(int t) { return static_cast<uint32_t>(t) * 128u; }
+  __device__ static constexpr uint32_t colO(int t) { return 256u + static_cast<uint32_t>(t) * D; }
+  static constexpr uint32_t kIdescS = idesc_bf16(kBM, kBN, 0, 0);
+  static constexpr uint32_t kIdescPV = idesc_bf16(kBM, D, 0, 1);
+};
+
+struct FwdBars {
+  uint64_t q_full;
+  uint64_t k_full[4], k_empty[4], v_full[4], v_empty[4];
+  uint64_t s_full[2], p_full[2], o_done[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+};
+
+// Wait on a barrier ignoring the CTA abort flag (used only to drain in-flight
+// MMAs before TMEM is released); still bounded.
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, unsigned long long limit_ns) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > limit_ns) break;
+  }
+}
+
+__device__ __forceinline__ bool warp_all(bool ok) { return __all_sync(0xffffffffu, ok); }
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                    const __grid_constant__ CUtensorMap tmV, const FwdArgs a, const DevCtl ctl) {
+  using C = FwdCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  FwdBars* bars = reinterpret_cast<FwdBars*>(smem + C::kOffBar);
+  const int warp = warp_id();
+  const int lane = lane_id();
+
+  // ---- work of this CTA ----
+  const int nqb = gridDim.x;
+  const int cb = a.causal ? (nqb - 1 - static_cast<int>(blockIdx.x)) : static_cast<int>(blockIdx.x);
+  const int h = blockIdx.y;
+  const int b = blockIdx.z;
+  const int nk_total = (a.N + kBN - 1) / kBN;
+  int q0[2], nkt[2];
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    q0[t] = cb * 2 * kBM + t * kBM;
+    nkt[t] = (q0[t] < a.N) ? (a.causal ? min(nk_total, q0[t] / kBN + 1) : nk_total) : 0;
+  }
+  const int nk = max(nkt[0], nkt[1]);
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars->q_full, 1);
+#pragma unroll
+    for (int s = 0; s < 4; ++s) {
+      mbar_init(&bars->k_full[s], 1);
+      mbar_init(&bars->k_empty[s], 1);
+      mbar_init(&bars->v_full[s], 1);
+      mbar_init(&bars->v_empty[s], 1);
+    }
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&bars->s_full[t], 1);
+      mbar_init(&bars->p_full[t], kBM);
+      mbar_init(&bars->o_done[t], 1);
+    }
+    mbar_init(&bars->drain, 1);
+    bars->abort = (*reinterpret_cast<volatile unsigned int*>(ctl.abort_epoch) == ctl.epoch) ? 1 : 0;
+    fence_mbar_init();
+  }
+  if (warp == 9) tmem_alloc(&bars->tmem_base, 512);
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+  const WaitCtl w{&bars->abort, ctl.status, ctl.abort_epoch, ctl.epoch, ctl.limit_ns};
+
+  if (warp < 8) {
+    reg_alloc<kRegSoftmax>();
+    if (bars->abort == 0) {
+      // ===================== softmax warps =====================
+      const int t = warp >> 2;
+      const int quarter = warp & 3;
+      const int r = quarter * 32 + lane;
+      const int qrow = q0[t] + r;
+      const uint32_t lane_bits = static_cast<uint32_t>(quarter * 32) << 16;
+      const uint32_t tS = tmem + lane_bits + C::colS(t);
+      const uint32_t tO = tmem + lane_bits + C::colO(t);
+      const float sl2 = a.scale_log2;
+      float m = -INFINITY;
+      float l = 0.f;
+      bool ok = true;
+      for (int j = 0; j < nkt[t]; ++j) {
+        ok = warp_all(wait_bar(&bars->s_full[t], j & 1, w, 8));
+        if (!ok) break;
+        tc_fence_after();
+        uint32_t sr[kBN];
+#pragma unroll
+        for (int c = 0; c < kBN / 32; ++c) tmem_ld32(tS + c * 32, sr + c * 32);
+        tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < kBN / 32; ++c) reg_fence32(sr + c * 32);
+
+        const int k0 = j * kBN;
+        const bool need_mask = (a.causal && k0 + kBN - 1 > q0[t]) || (k0 + kBN > a.N);
+        if (need_mask) {
+          const int lim = a.causal ? min(a.N - 1, qrow) : (a.N - 1);  // last visible key
+#pragma unroll
+          for (int c = 0; c < kBN; ++c)
+            if (k0 + c > lim) sr[c] = __float_as_uint(-INFINITY);
+        }
+        float mx0 = __uint_as_float(sr[0]), mx1 = __uint_as_float(sr[1]);
+        float mx2 = __uint_as_float(sr[2]), mx3 = __uint_as_float(sr[3]);
+#pragma unroll
+        for (int c = 4; c < kBN; c += 4) {
+          mx0 = fmaxf(mx0, __uint_as_float(sr[c + 0]));
+          mx1 = fmaxf(mx1, __uint_as_float(sr[c + 1]));
+          mx2 = fmaxf(mx2, __uint_as_float(sr[c + 2]));
+          mx3 = fmaxf(mx3, __uint_as_float(sr[c + 3]));
+        }
+        const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+        const float m_new = fmaxf(m, mx * sl2);
+        const bool need = m_new > m + kTau;
+        if (__any_sync(0xffffffffu, need)) {
+          const float alpha = (m_new == -INFINITY) ? 1.f : ex2(m - m_new);
+          l *= alpha;
+          if (j > 0) {
+            // O_t holds the sum over the previous key tiles; PV of tile j-1
+            // completed before S_t of tile j was issued.
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+              uint32_t o[32];
+              tmem_ld32(tO + c * 32, o);
+              tmem_wait_ld();
+              reg_fence32(o);
+#pragma unroll
+              for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+              tmem_st32(tO + c * 32, o);
+            }
+          }
+          m = m_new;
+        }
+        const float neg_m = (m == -INFINITY) ? 0.f : -m;
+        float rs0 = 0.f, rs1 = 0.f;
+        // P_t (bf16, two per column) over the first 64 columns of S_t, written
+        // 32 columns at a time
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+          uint32_t pk[32];
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            const float p0 = ex2(fmaf(__uint_as_float(sr[64 * h2 + 2 * c]), sl2, neg_m));
+            const float p1 = ex2(fmaf(__uint_as_float(sr[64 * h2 + 2 * c + 1]), sl2, neg_m));
+            rs0 += p0;
+            rs1 += p1;
+            pk[c] = pack_bf16x2(p0, p1);
+          }
+          tmem_st32(tS + 32 * h2, pk);
+        }
+        l += rs0 + rs1;
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&bars->p_full[t]);
+      }
+      // ---- epilogue ----
+      if (ok && nkt[t] > 0) {
+        ok = warp_all(wait_bar(&bars->o_done[t], (nkt[t] - 1) & 1, w, 9));
+        if (ok) {
+          tc_fence_after();
+          const float inv = (l > 0.f) ? 1.f / l : 0.f;
+          __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.O) +
+                                ((static_cast<size_t>(b) * a.N + qrow) * a.H + h) * D;
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t o[32];
+            tmem_ld32(tO + c * 32, o);
+            tmem_wait_ld();
+            reg_fence32(o);
+            uint32_t pkd[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              pkd[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
+            if (qrow < a.N) {
+#pragma unroll
+              for (int i = 0; i < 4; ++i)
+                st_global_v4(orow + c * 32 + i * 8, pkd[4 * i], pkd[4 * i + 1], pkd[4 * i + 2], pkd[4 * i + 3]);
+            }
+          }
+          if (qrow < a.N) {
+            const float lse = (l > 0.f) ? (m + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+            a.LSE[(static_cast<size_t>(b) * a.H + h) * a.N + qrow] = lse;
+          }
+        }
+      }
+    }
+  } else {
+    reg_dealloc<kRegOther>();
+    if (bars->abort == 0 && warp == 8) {
+      // ===================== TMA producer =====================
+      if (lane == 0) {
+        tma_prefetch_desc(&tmQ);
+        tma_prefetch_desc(&tmK);
+        tma_prefetch_desc(&tmV);
+        uint32_t qbytes = 0;
+        for (int t = 0; t < 2; ++t) qbytes += (nkt[t] > 0) ? C::kTileBytes : 0;
+        mbar_arrive_expect_tx(&bars->q_full, qbytes);
+        for (int t = 0; t < 2; ++t) {
+          if (nkt[t] == 0) continue;
+          for (int c = 0; c < C::kSub; ++c)
+            tma_load_4d(smem + C::kOffQ + t * C::kTileBytes + c * C::kSubBytes, &tmQ, &bars->q_full, c * 64,
+                        q0[t], h, b);
+        }
+        for (int j = 0; j < nk; ++j) {
+          const int s = j % C::kStages;
+          const int n = j / C::kStages;
+          if (j >= C::kStages && !wait_bar(&bars->k_empty[s], (n - 1) & 1, w, 1)) break;
+          const uint32_t extra = (ctl.inject == 1 && j == 0) ? 16u : 0u;  // test-only: never completes
+          mbar_arrive_expect_tx(&bars->k_full[s], C::kTileBytes + extra);
+          for (int c = 0; c < C::kSub; ++c)
+            tma_load_4d(smem + C::kOffK + s * C::kTileBytes + c * C::kSubBytes, &tmK, &bars->k_full[s], c * 64,
+                        j * kBN, h, b);
+          if (j >= C::kStages && !wait_bar(&bars->v_empty[s], (n - 1) & 1, w, 2)) break;
+          mbar_arrive_expect_tx(&bars->v_full[s], C::kTileBytes);
+          for (int c = 0; c < C::kSub; ++c)
+            tma_load_4d(smem + C::kOffV + s * C::kTileBytes + c * C::kSubBytes, &tmV, &bars->v_full[s], c * 64,
+                        j * kBN, h, b);
+        }
+      }
+    } else if (warp == 9) {
+      // ===================== MMA issuer (one thread) =====================
+      if (lane == 0) {
+        const uint32_t sQ = smem_u32(smem + C::kOffQ);
+        const uint32_t sK = smem_u32(smem + C::kOffK);
+        const uint32_t sV = smem_u32(smem + C::kOffV);
+        bool ok = wait_bar(&bars->q_full, 0, w, 3);
+        for (int j = 0; ok && j < nk; ++j) {
+          const int s = j % C::kStages;
+          const uint32_t ph = (j / C::kStages) & 1;
+          if (!(ok = wait_bar(&bars->k_full[s], ph, w, 4))) break;
+          tc_fence_after();
+          for (int t = 0; t < 2; ++t) {
+            if (j >= nkt[t]) continue;
+            // S_t is overwritten: the previous P_t must have been consumed.
+            if (j > 0 && !(ok = wait_bar(&bars->o_done[t], (j - 1) & 1, w, 5))) break;
+            tc_fence_after();
+            const uint32_t qa = sQ + t * C::kTileBytes;
+            const uint32_t kb = sK + s * C::kTileBytes;
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t off = (kk >> 2) * C::kSubBytes + (kk & 3) * 32;
+              umma_ss(tmem + C::colS(t), sw128_desc(qa + off, 16, 1024), sw128_desc(kb + off, 16, 1024),
+                      C::kIdescS, kk > 0 ? 1u : 0u);
+            }
+            umma_commit(&bars->s_full[t]);
+          }
+          if (!ok) break;
+          umma_commit(&bars->k_empty[s]);
+          if (!(ok = wait_bar(&bars->v_full[s], ph, w, 6))) break;
+          tc_fence_after();
+          for (int t = 0; t < 2; ++t) {
+            if (j >= nkt[t]) continue;
+            if (!(ok = wait_bar(&bars->p_full[t], j & 1, w, 7))) break;
+            tc_fence_after();
+            const uint32_t vb = sV + s * C::kTileBytes;
+#pragma unroll
+            for (int kk = 0; kk < kBN / 16; ++kk) {
+              umma_ts(tmem + C::colO(t), tmem + C::colS(t) + kk * 8,
+                      sw128_desc(vb + kk * 2048, C::kSubBytes, 1024), C::kIdescPV,
+                      (j > 0 || kk > 0) ? 1u : 0u);
+            }
+            umma_commit(&bars->o_done[t]);
+          }
+          if (!ok) break;
+          umma_commit(&bars->v_empty[s]);
+        }
+        // all MMAs of this CTA finish before TMEM is released
+        umma_commit(&bars->drain);
+        drain_wait(&bars->drain, 0, ctl.limit_ns);
+      }
+    }
+  }
+
+  // ---- teardown ----
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_fwd_bf16(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const FwdArgs& a,
+                            const DevCtl& c, cudaStream_t s) {
+  const int nqb = (a.N + 2 * kBM - 1) / (2 * kBM);
+  const dim3 grid(nqb, a.H, a.B);
+  if (a.d == 128) {
+    constexpr int smem = FwdCfg<128>::kSmemBytes;
+    cudaError_t e = cudaFuncSetAttribute(fwd_bf16_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    fwd_bf16_kernel<128><<<grid, kThreads, smem, s>>>(tq, tk, tv, a, c);
+  } else {
+    constexpr int smem = FwdCfg<64>::kSmemBytes;
+    cudaError_t e = cudaFuncSetAttribute(fwd_bf16_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    fwd_bf16_kernel<64><<<grid, kThreads, smem, s>>>(tq, tk, tv, a, c);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace fa

@@ -1,0 +1,62 @@
+// Internal (not exported) declarations shared by the host library and the
+// kernel translation units.  Nothing here is part of the C ABI.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace fa {
+
+// Device-side error reporting for one launch.
+struct DevCtl {
+  int* status;                  // device status word (0 = ok)
+  unsigned int* abort_epoch;    // epoch of the last launch that hit a wait limit
+  unsigned int epoch;           // epoch of this launch
+  unsigned long long limit_ns;  // limit for any single wait
+  int inject;                   // test-only fault injection (0 = off)
+};
+
+struct FwdArgs {
+  int B, H, N, d;
+  float scale_log2;  // softmax scale * log2(e)
+  int causal;
+  void* O;           // [B, N, H, d]
+  float* LSE;        // [B, H, N], natural log
+};
+
+struct BwdArgs {
+  int B, H, N, d, Npad;
+  float scale;       // softmax scale
+  float scale_log2;  // scale * log2(e)
+  int causal;
+  const void* O;
+  const void* dO;
+  const float* LSE;  // [B, H, N] natural log
+  void* dQ;
+  void* dK;
+  void* dV;
+  float* dQacc;      // [B, N, H, d] fp32 workspace
+  float* Dvec;       // [B, H, Npad] rowsum(dO * O)
+  float* LSE2;       // [B, H, Npad] LSE * log2(e)
+};
+
+// TMA descriptor for a [B, N, H, d] bf16 tensor with a box of `rows` sequence
+// positions x 64 features of one (b, h); 128-byte swizzle.
+CUresult make_tile_map(CUtensorMap* map, const void* base, int B, int N, int H, int d, int rows);
+
+// Kernel launchers (each returns the cudaError_t of the launch).
+cudaError_t launch_fwd_bf16(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                            const FwdArgs& a, const DevCtl& c, cudaStream_t s);
+cudaError_t launch_fwd_f32(const float* Q, const float* K, const float* V, const FwdArgs& a, cudaStream_t s);
+cudaError_t launch_bwd_pre(const BwdArgs& a, cudaStream_t s);
+cudaError_t launch_bwd_main(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                            const CUtensorMap& tdo, const BwdArgs& a, const DevCtl& c, cudaStream_t s);
+cudaError_t launch_bwd_dq(const BwdArgs& a, cudaStream_t s);
+
+// Test-only single-tile MMA probe (see fa_debug_umma in the public header).
+cudaError_t launch_umma_probe(const void* A, const void* B, float* D, int N, int K, int a_mn_major,
+                              int b_mn_major, int a_tmem, cudaStream_t s);
+
+}  // namespace fa

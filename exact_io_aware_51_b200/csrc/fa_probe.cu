@@ -1,0 +1,131 @@
+// Test-only probe of one tcgen05 MMA tile: D[128][N] = A[128][K] * B[N][K]^T.
+//
+// It checks, on its own, each operand layout the attention kernels hand to the
+// tensor cores: 128-byte swizzled K-major and MN-major shared-memory operands,
+// and A read from tensor memory.  The threads place A and B in shared memory
+// with the same swizzle the TMA produces, one thread issues the MMAs, and the
+// fp32 result is read back through tcgen05.ld.
+#include <cuda_bf16.h>
+
+#include "fa_internal.h"
+#include "sm100.cuh"
+
+namespace fa {
+namespace {
+
+__global__ void __launch_bounds__(128, 1)
+    umma_probe_kernel(const __nv_bfloat16* __restrict__ A, const __nv_bfloat16* __restrict__ B, float* __restrict__ D,
+                      int N, int K, int a_mn, int b_mn, int a_tmem) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;                 // up to 128 x 128 bf16 = 32 KB
+  uint8_t* sB = smem + 32768;         // up to 128 x 128 bf16 = 32 KB
+  __shared__ uint64_t bar;
+  __shared__ uint32_t tbase;
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+
+  // ---- A into shared memory ----
+  for (int e = tid; e < 128 * K; e += 128) {
+    const int m = e / K, k = e % K;
+    uint32_t off;
+    if (a_mn == 0)
+      off = (k / 64) * (128 * 128) + sw128_offset(m, (k % 64) / 8) + (k % 8) * 2;
+    else
+      off = (m / 64) * (K * 128) + sw128_offset(k, (m % 64) / 8) + (m % 8) * 2;
+    *reinterpret_cast<__nv_bfloat16*>(sA + off) = A[e];
+  }
+  // ---- B into shared memory ----
+  for (int e = tid; e < N * K; e += 128) {
+    const int n = e / K, k = e % K;
+    uint32_t off;
+    if (b_mn == 0)
+      off = (k / 64) * (N * 128) + sw128_offset(n, (k % 64) / 8) + (k % 8) * 2;
+    else
+      off = (n / 64) * (K * 128) + sw128_offset(k, (n % 64) / 8) + (n % 8) * 2;
+    *reinterpret_cast<__nv_bfloat16*>(sB + off) = B[e];
+  }
+  if (tid == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) tmem_alloc(&tbase, 512);
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tbase;
+  const uint32_t lane_bits = static_cast<uint32_t>(warp * 32) << 16;
+
+  if (a_tmem) {
+    // row m = tid into lane m, two bf16 per column starting at column 256
+    for (int c0 = 0; c0 < K / 2; c0 += 16) {
+      uint32_t r[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int k = 2 * (c0 + i);
+        const __nv_bfloat162 v = __halves2bfloat162(A[tid * K + k], A[tid * K + k + 1]);
+        r[i] = *reinterpret_cast<const uint32_t*>(&v);
+      }
+      tmem_st16(tmem + lane_bits + 256 + c0, r);
+    }
+    tmem_wait_st();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+  }
+
+  if (tid == 0) {
+    const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sB);
+    const uint32_t idesc = idesc_bf16(128, N, a_tmem ? 0 : a_mn, b_mn);
+    for (int kk = 0; kk < K / 16; ++kk) {
+      const uint64_t bd = (b_mn == 0) ? sw128_desc(b0 + (kk / 4) * (N * 128) + (kk % 4) * 32, 16, 1024)
+                                      : sw128_desc(b0 + kk * 2048, K * 128, 1024);
+      if (a_tmem) {
+        umma_ts(tmem, tmem + 256 + kk * 8, bd, idesc, kk > 0 ? 1u : 0u);
+      } else {
+        const uint64_t ad = (a_mn == 0) ? sw128_desc(a0 + (kk / 4) * (128 * 128) + (kk % 4) * 32, 16, 1024)
+                                        : sw128_desc(a0 + kk * 2048, K * 128, 1024);
+        umma_ss(tmem, ad, bd, idesc, kk > 0 ? 1u : 0u);
+      }
+    }
+    umma_commit(&bar);
+  }
+  // bounded wait for the MMAs (no other role can stall this one)
+  const uint64_t t0 = globaltimer_ns();
+  bool done = false;
+  while (!(done = mbar_try_wait(&bar, 0)) && globaltimer_ns() - t0 < 2000000000ull) {
+  }
+  done = __all_sync(0xffffffffu, done);
+  tc_fence_after();
+  if (done) {
+    for (int c0 = 0; c0 < N; c0 += 32) {
+      uint32_t r[32];
+      tmem_ld32(tmem + lane_bits + c0, r);
+      tmem_wait_ld();
+      reg_fence32(r);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) D[tid * N + c0 + i] = __uint_as_float(r[i]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_umma_probe(const void* A, const void* B, float* D, int N, int K, int a_mn, int b_mn, int a_tmem,
+                              cudaStream_t s) {
+  constexpr int smem = 65536 + 1024;
+  cudaError_t e = cudaFuncSetAttribute(umma_probe_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  umma_probe_kernel<<<1, 128, smem, s>>>(static_cast<const __nv_bfloat16*>(A), static_cast<const __nv_bfloat16*>(B),
+                                         D, N, K, a_mn, b_mn, a_tmem);
+  return cudaGetLastError();
+}
+
+}  // namespace fa

@@ -1,0 +1,166 @@
+/*
+ * Exact IO-aware attention on B200 (sm_100a): the C ABI.
+ *
+ * What the library computes (per batch b and head h):
+ *
+ *     S = scale * Q K^T  (+ causal mask: key j hidden from query i when j > i)
+ *     O = softmax_rows(S) V,      LSE_i = log sum_j exp(S_ij)   (natural log)
+ *
+ * exactly as standard attention does, without ever writing the N x N score
+ * matrix to device memory.  Sources (web pages on FlashAttention, cited by
+ * title and section):
+ *   "Flash Attention" (karlkratz.de): "Tiling: Blockweise Berechnung im
+ *     schnellen Speicher" (block-wise computation with a running maximum and
+ *     sum per row), "Speicherbedarf und Laufzeitverhalten" (O(N) extra memory,
+ *     exactly the same result), "Recomputation beim Rückwärtsdurchlauf"
+ *     (the backward pass recomputes the attention values).
+ *   "Flash Attention" (Ultralytics glossary): "Принцип работы Flash Attention"
+ *     (query block resident, key/value blocks streamed, only the output and
+ *     per-row statistics return to HBM; backward recomputes score blocks).
+ *   "Beschleunigte Transformer: FlashAttention, effiziente Kernel und kluge
+ *     Speicherlayouts": "Layout-Entscheidungen für Q, K und V" (the
+ *     [batch, sequence, heads, features] layout used here).
+ *
+ * Conventions shared by every entry point
+ *   Layout: Q, K, V, O, dO, dQ, dK, dV are dense, contiguous [B, N, H, d]
+ *     tensors (element (b, n, h, k) at ((b*N + n)*H + h)*d + k) of the call's
+ *     dtype.  LSE is a dense [B, H, N] fp32 tensor in natural-log units.
+ *   Pointers: all tensor pointers are DEVICE pointers of the current CUDA
+ *     device and must be 16-byte aligned.  The caller allocates and owns every
+ *     buffer, including the backward workspace.  The library allocates no
+ *     device memory, copies nothing between host and device and never
+ *     synchronises, except where an entry point says so.
+ *   Stream: `stream` is a cudaStream_t (NULL = the legacy default stream).
+ *     All work is enqueued asynchronously on it.
+ *   Sizes: B, H, N >= 0; B*H*N == 0 is a valid empty problem (returns FA_OK,
+ *     writes nothing).  d must be 64 or 128.  N <= 2^22, H <= 65535,
+ *     B <= 65535.
+ *   Errors: every entry point returns 0 (FA_OK) or a negative FA_ERR_* code;
+ *     on a validation error nothing is enqueued and no output is written.
+ *     An unsupported shape is refused rather than computed wrongly (a wrongly
+ *     configured block size "leads to errors": "Flash Attention"
+ *     (karlkratz.de), "Grenzen und Einschränkungen").
+ *   Threads: entry points are safe to call from several host threads.
+ */
+#ifndef EXACT_IO_AWARE_FA_H
+#define EXACT_IO_AWARE_FA_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Element type of Q, K, V, O, dO, dQ, dK, dV. */
+typedef enum { FA_BF16 = 0, FA_FP32 = 1 } fa_dtype;
+
+enum {
+  FA_OK = 0,
+  FA_ERR_INVALID_ARG = -1,     /* null pointer, negative size, bad scale or dtype */
+  FA_ERR_UNSUPPORTED = -2,     /* d not 64/128, or a dtype/d the pass does not implement */
+  FA_ERR_MISALIGNED = -3,      /* a tensor pointer is not 16-byte aligned */
+  FA_ERR_WORKSPACE = -4,       /* backward workspace missing, too small or misaligned */
+  FA_ERR_ARCH = -5,            /* current device is not compute capability 10.0 */
+  FA_ERR_LAUNCH = -6,          /* a CUDA call failed; see fa_last_cuda_error() */
+  FA_ERR_DEVICE_TIMEOUT = -7,  /* a kernel's bounded wait expired (see fa_last_device_status) */
+  FA_ERR_TOO_LARGE = -8        /* a size limit above is exceeded */
+};
+
+/*
+ * Forward pass.
+ *   Q, K, V  [B, N, H, d] inputs (dtype).
+ *   O        [B, N, H, d] output (dtype), written completely.
+ *   LSE      [B, H, N] fp32 output, natural log of the softmax denominator
+ *            of each row (the one per-row statistic the backward needs).
+ *   scale    softmax scale, finite and > 0 (usually 1/sqrt(d)).
+ *   causal   0 = bidirectional, 1 = key j hidden from query i when j > i.
+ *   dtype    FA_BF16: tcgen05 tensor-core kernel, fp32 accumulation, O in bf16.
+ *            FA_FP32: fp32 CUDA-core kernel (no TF32), O in fp32.
+ * Online softmax over streamed key/value tiles ("Flash Attention" (Ultralytics
+ * glossary), "Принцип работы Flash Attention"); only O and LSE reach memory.
+ */
+int fa_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, int B, int H, int N, int d,
+           float scale, int causal, int dtype, void* stream);
+
+/*
+ * Bytes of device workspace fa_bwd needs for this problem: an fp32 dQ
+ * accumulator [B, N, H, d] plus two fp32 [B, H, roundup(N, 128)] rows
+ * (rowsum(dO * O) and LSE * log2 e), each region 256-byte aligned.  This is
+ * the O(N) extra memory of the method ("Flash Attention" (karlkratz.de),
+ * "Speicherbedarf und Laufzeitverhalten").  Returns 0 for invalid or empty
+ * problems.
+ */
+size_t fa_bwd_workspace_size(int B, int H, int N, int d, int dtype);
+
+/*
+ * Backward pass by recomputation ("Flash Attention" (karlkratz.de),
+ * "Recomputation beim Rückwärtsdurchlauf"): score tiles are rebuilt from Q, K
+ * and the saved LSE, and
+ *   dV = P^T dO, dP = dO V^T, D_i = sum_k dO_ik O_ik, dS = P * (dP - D),
+ *   dQ = scale * dS K, dK = scale * dS^T Q.
+ *   Q, K, V, O, dO  [B, N, H, d] inputs; O and LSE as written by fa_fwd.
+ *   dQ, dK, dV      [B, N, H, d] outputs, written completely.
+ *   workspace       device buffer of at least fa_bwd_workspace_size() bytes,
+ *                   256-byte aligned; overwritten.
+ * Currently dtype FA_BF16 with d = 128 (FA_ERR_UNSUPPORTED otherwise).
+ * dQ is accumulated with fp32 atomics, so it is not bitwise deterministic.
+ */
+int fa_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO, const float* LSE, void* dQ,
+           void* dK, void* dV, int B, int H, int N, int d, float scale, int causal, int dtype, void* workspace,
+           size_t workspace_bytes, void* stream);
+
+/* Static English text for a status code. */
+const char* fa_status_string(int status);
+
+/* The cudaError_t of the last failed CUDA call on this host thread (0 if none);
+ * 100000 + CUresult when encoding a TMA descriptor failed. */
+int fa_last_cuda_error(void);
+
+/*
+ * Synchronises `stream`, then reads and clears the current device's status
+ * word.  Returns FA_OK if no kernel reported a problem since the last call,
+ * FA_ERR_DEVICE_TIMEOUT if a bounded wait expired (the affected launch's
+ * outputs are then undefined), or FA_ERR_LAUNCH.  *detail (if not NULL)
+ * receives the raw word: 0x1000 | the id of the wait that expired.
+ */
+int fa_last_device_status(void* stream, int* detail);
+
+/*
+ * Test and diagnostics knobs (process-wide).
+ *   fa_set_wait_limit_ms: limit for any single wait inside a kernel
+ *     (default 2000 ms, or the FA_TIMEOUT_MS environment variable).
+ *   fa_debug_inject: 1 makes the next forward launches' first key-tile
+ *     barrier expect 16 bytes that never arrive, so its waits expire and the
+ *     launch reports FA_ERR_DEVICE_TIMEOUT; 0 turns it off.
+ */
+void fa_set_wait_limit_ms(int ms);
+void fa_debug_inject(int mode);
+
+/*
+ * Diagnostics: while set, each fa_fwd / fa_bwd call made on this host thread
+ * records the cudaEvent_t `start` on its stream right before its tensor-core
+ * kernel (the fused forward, or the backward main kernel) and `stop` right
+ * after it, so a caller can time that one kernel with cudaEventElapsedTime.
+ * Pass NULL, NULL to turn it off.  The events stay owned by the caller.
+ */
+void fa_set_kernel_events(void* start, void* stop);
+
+/*
+ * Test-only: one 128 x N x K tcgen05 MMA tile, D = A B^T, with A [128][K] and
+ * B [N][K] bf16 row-major device arrays and D [128][N] fp32.  a_mn_major /
+ * b_mn_major choose how the operand is laid out in shared memory (0: the
+ * reduction dimension contiguous, 1: the M or N dimension contiguous); a_tmem
+ * reads A from tensor memory instead.  N and K must be 64 or 128.  Synchronous
+ * on `stream` is not implied.
+ */
+int fa_debug_umma(const void* A, const void* B, float* D, int N, int K, int a_mn_major, int b_mn_major,
+                  int a_tmem, void* stream);
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+int fa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EXACT_IO_AWARE_FA_H */

@@ -1,0 +1,112 @@
+"""Library loading, exported symbols and host-side validation (no GPU work).
+
+Every call here is rejected by the host-side checks before any CUDA call, or
+reads only static data, so it runs on a machine without a GPU.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import pathlib
+import re
+import subprocess
+
+import pytest
+
+import exact_io_aware_51_b200 as fa
+from exact_io_aware_51_b200 import build as fabuild
+
+ROOT = pathlib.Path(__file__).resolve().parents[1]
+HEADER = ROOT / "include" / "fa.h"
+
+
+@pytest.fixture(scope="module")
+def L():
+    fabuild.build()
+    return fa.lib()
+
+
+def declared_functions():
+    text = HEADER.read_text()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(fa_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_what_the_binding_lists():
+    assert declared_functions() == sorted(fa.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol(L):
+    out = subprocess.run(["nm", "-D", "--defined-only", str(fa.lib_path())], capture_output=True, text=True,
+                         check=True).stdout
+    exported = set(re.findall(r" T (fa_[a-z0-9_]+)$", out, flags=re.M))
+    for name in declared_functions():
+        assert name in exported, name
+        assert getattr(L, name) is not None
+
+
+def test_status_strings(L):
+    for code in (0, -1, -2, -3, -4, -5, -6, -7, -8):
+        assert fa.status_string(code) and "unknown" not in fa.status_string(code)
+    assert "unknown" in fa.status_string(-99)
+
+
+def test_validation_rejects_before_touching_the_device(L):
+    f = L.fa_fwd
+    # null pointers
+    assert f(None, None, None, None, None, 1, 1, 128, 64, 0.125, 0, 0, None) == -1
+    # unsupported head dim
+    assert f(16, 16, 16, 16, 16, 1, 1, 128, 96, 0.125, 0, 0, None) == -2
+    # negative sizes, bad dtype, bad scale
+    assert f(16, 16, 16, 16, 16, -1, 1, 128, 64, 0.125, 0, 0, None) == -1
+    assert f(16, 16, 16, 16, 16, 1, 1, 128, 64, 0.125, 0, 7, None) == -1
+    for bad in (0.0, -1.0, float("inf"), float("nan")):
+        assert f(16, 16, 16, 16, 16, 1, 1, 128, 64, bad, 0, 0, None) == -1
+    # misaligned pointer
+    assert f(8, 16, 16, 16, 16, 1, 1, 128, 64, 0.125, 0, 0, None) == -3
+    # size limits
+    assert f(16, 16, 16, 16, 16, 1, 1, (1 << 22) + 1, 64, 0.125, 0, 0, None) == -8
+    assert f(16, 16, 16, 16, 16, 1, 65536, 128, 64, 0.125, 0, 0, None) == -8
+    # empty problems are valid no-ops
+    assert f(None, None, None, None, None, 0, 4, 128, 64, 0.125, 0, 0, None) == 0
+    assert f(None, None, None, None, None, 2, 4, 0, 64, 0.125, 0, 0, None) == 0
+
+
+def test_backward_validation(L):
+    b = L.fa_bwd
+    args = [16] * 9
+    ws = L.fa_bwd_workspace_size(1, 1, 128, 128, 0)
+    # fp32 backward and d = 64 backward are not implemented: refused
+    assert b(*args, 1, 1, 128, 128, 0.1, 0, 1, 256, ws, None) == -2
+    assert b(*args, 1, 1, 128, 64, 0.1, 0, 0, 256, ws, None) == -2
+    # workspace missing / too small / misaligned
+    assert b(*args, 1, 1, 128, 128, 0.1, 0, 0, None, ws, None) == -4
+    assert b(*args, 1, 1, 128, 128, 0.1, 0, 0, 256, ws - 1, None) == -4
+    assert b(*args, 1, 1, 128, 128, 0.1, 0, 0, 272, ws, None) == -4
+    # misaligned tensor
+    bad = list(args)
+    bad[7] = 24
+    assert b(*bad, 1, 1, 128, 128, 0.1, 0, 0, 256, ws, None) == -3
+
+
+def test_workspace_is_linear_in_n(L):
+    """The method's extra memory is O(N): the fp32 dQ accumulator plus two rows per (b, h)."""
+    def ws(n):
+        return L.fa_bwd_workspace_size(2, 16, n, 128, 0)
+    B, H, d = 2, 16, 128
+    for n in (128, 4096, 16384):
+        expect = B * n * H * d * 4 + 2 * B * H * n * 4
+        assert ws(n) == expect
+    # versus the N x N score matrix standard attention would store (2 bytes each)
+    assert ws(16384) < 2 * 16384 * 16384 * H * B
+    assert L.fa_bwd_workspace_size(0, 1, 1, 128, 0) == 0
+    assert L.fa_bwd_workspace_size(1, 1, 1, 96, 0) == 0
+    # ragged N rounds the per-row arrays up to a multiple of 128
+    assert ws(130) == ((2 * 130 * 16 * 128 * 4 + 255) // 256 * 256) + 2 * ((2 * 16 * 256 * 4 + 255) // 256 * 256)
+
+
+def test_python_binding_refuses_cpu_tensors(L):
+    import torch
+    q = torch.zeros(1, 128, 1, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA"):
+        fa.fwd(q, q, q)
