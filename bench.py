@@ -156,6 +156,21 @@ def head_inputs(seed=0):
     return tuple(t[0, :, 0].float().numpy().astype(np.float64) for t in (q, k, v, do))
 
 
+def max_over_ranks(x: float, dist=None, device=None) -> float:
+    """The slowest rank's value (all ranks take part; a no-op without a process group)."""
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return x
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_tflops(flops_per_rank_step: float, steps: int, world: int, ms_max: float) -> float:
+    """Whole-job throughput: every rank's FLOPs over the slowest rank's time."""
+    return flops_per_rank_step * steps * world / (ms_max * 1e-3) / 1e12
+
+
 def dist_setup(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -223,12 +238,8 @@ def run_ours(args, world, rank, local):
         if dist is not None:
             dist.barrier()
 
-    def max_over_ranks(x: float) -> float:
-        if dist is None:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    def slowest(x: float) -> float:
+        return max_over_ranks(x, dist, dev)
 
     for _ in range(args.warmup):
         step()
@@ -237,8 +248,15 @@ def run_ours(args, world, rank, local):
     sampler = ClockSampler(local)
     sampler.start()
     # ---- timed region: K steps, kernel events around the two tensor-core kernels ----
-    ev_f = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    ev_b = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    def kernel_event():
+        # torch creates the CUDA event lazily on its first record; record it once
+        # here so the handle exists when the library records it around a kernel
+        e = torch.cuda.Event(enable_timing=True)
+        e.record(stream)
+        return e
+
+    ev_f = [(kernel_event(), kernel_event()) for _ in range(args.steps)]
+    ev_b = [(kernel_event(), kernel_event()) for _ in range(args.steps)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize()
@@ -257,13 +275,12 @@ def run_ours(args, world, rank, local):
     if rc != 0:
         raise RuntimeError(f"device status {rc} ({detail:#x}) after the timed region")
     ms_local = t0.elapsed_time(t1)
-    ms = max_over_ranks(ms_local)
-    fwd_ms = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in ev_f))
-    bwd_main_ms = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in ev_b))
+    ms = slowest(ms_local)
+    fwd_ms = slowest(statistics.mean(a.elapsed_time(b) for a, b in ev_f))
+    bwd_main_ms = slowest(statistics.mean(a.elapsed_time(b) for a, b in ev_b))
 
     f = flops_fwd(B, H, N, d, causal)
-    total_flops = 3.5 * f * args.steps * world
-    value = total_flops / (ms * 1e-3) / 1e12
+    value = aggregate_tflops(3.5 * f, args.steps, world, ms)
     ms_step = ms / args.steps
     peak_burst, peak_sustained, peak_src = read_peaks()
     fwd_tflops = f / (fwd_ms * 1e-3) / 1e12
@@ -305,8 +322,8 @@ def run_ours(args, world, rank, local):
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1))
-    e2e_value = 3.5 * f * e_steps * world / (e2e_ms * 1e-3) / 1e12
+    e2e_ms = slowest(e0.elapsed_time(e1))
+    e2e_value = aggregate_tflops(3.5 * f, e_steps, world, e2e_ms)
 
     result = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,

@@ -25,6 +25,7 @@ constexpr int kMaxDevices = 64;
 constexpr long long kMaxN = 1LL << 22;
 
 thread_local int t_last_cuda_error = 0;
+thread_local int t_bound_device = -1;  // device whose primary context this thread has made current
 thread_local cudaEvent_t t_ev_start = nullptr;
 thread_local cudaEvent_t t_ev_stop = nullptr;
 std::atomic<unsigned int> g_epoch{1};
@@ -73,6 +74,14 @@ int device_state(DeviceState** out) {
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return fail_cuda(e);
   if (dev < 0 || dev >= kMaxDevices) return FA_ERR_ARCH;
+  // A thread that has not yet made a CUDA runtime call that needs a context
+  // (for example an autograd worker thread) has none current; the driver's TMA
+  // descriptor encoder needs one, so bind the device's primary context once.
+  if (t_bound_device != dev) {
+    e = cudaSetDevice(dev);
+    if (e != cudaSuccess) return fail_cuda(e);
+    t_bound_device = dev;
+  }
   DeviceState& st = g_dev[dev];
   std::call_once(st.once, [&] {
     int major = 0, minor = 0;

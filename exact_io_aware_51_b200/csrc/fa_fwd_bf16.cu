@@ -42,6 +42,32 @@ constexpr int kThreads = 384;   // WG0, WG1: softmax; WG2: loader warp, MMA warp
 constexpr uint32_t kRegSoftmax = 216;
 constexpr uint32_t kRegOther = 72;
 constexpr float kTau = 8.0f;    // lazy-rescale threshold (log2 units)
+// When > 0, one score pair in kPolyEvery takes its exponentials on the FMA pipe
+// (exp2_poly2) instead of the MUFU unit.  Measured on B200 at d = 128 the MUFU
+// is not what limits this kernel (1/4, 1/3 and 1/2 of the pairs on the FMA pipe
+// were 6-10% slower than none), so it is off.
+constexpr int kPolyEvery = 0;
+
+// 2^x for a pair on the FMA/ALU pipes: x = n + f with n = round(x) (taken by
+// adding and subtracting 1.5 * 2^23) and f in [-1/2, 1/2]; 2^f from a degree-3
+// polynomial with minimal maximum relative error (7.5e-5) on that interval,
+// fitted by the Remez exchange algorithm in gen_exp2_poly.py; 2^n is added to
+// the exponent bits.  x is clamped below at -125 (2^-125 is zero for P after
+// the bf16 rounding), which also maps -inf (masked scores) to that floor.
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
+  x.x = fmaxf(x.x, -125.f);
+  x.y = fmaxf(x.y, -125.f);
+  const float2 t = fadd2(x, make_float2(kShift, kShift));
+  const float2 n = fadd2(t, make_float2(-kShift, -kShift));
+  const float2 f = fadd2(x, make_float2(-n.x, -n.y));
+  float2 p = ffma2(make_float2(5.517166853e-02f, 5.517166853e-02f), f, make_float2(2.426111251e-01f, 2.426111251e-01f));
+  p = ffma2(p, f, make_float2(6.932609677e-01f, 6.932609677e-01f));
+  p = ffma2(p, f, make_float2(9.999280572e-01f, 9.999280572e-01f));
+  const uint32_t ex = __float_as_uint(t.x) << 23;
+  const uint32_t ey = __float_as_uint(t.y) << 23;
+  return make_float2(__uint_as_float(__float_as_uint(p.x) + ex), __uint_as_float(__float_as_uint(p.y) + ey));
+}
 
 template <int D>
 struct FwdCfg {
@@ -181,8 +207,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float alpha = (m_new == -INFINITY) ? 1.f : ex2(m - m_new);
           l *= alpha;
           if (j > 0) {
-            // O_t holds the sum over the previous key tiles; PV of tile j-1
-            // completed before S_t of tile j was issued.
+            // O_t holds the sum over the previous key tiles: PV_t(j-1) was
+            // issued before S_t(j), and s_full fired when S_t(j) completed.
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) {
               uint32_t o[32];
@@ -197,23 +223,31 @@ __global__ void __launch_bounds__(kThreads, 1)
           m = m_new;
         }
         const float neg_m = (m == -INFINITY) ? 0.f : -m;
-        float rs0 = 0.f, rs1 = 0.f;
+        const float2 sl2v = make_float2(sl2, sl2);
+        const float2 negmv = make_float2(neg_m, neg_m);
+        float2 rs = make_float2(0.f, 0.f);
         // P_t (bf16, two per column) over the first 64 columns of S_t, written
-        // 32 columns at a time
+        // 16 columns (32 scores) at a time so the stores overlap the math
 #pragma unroll
-        for (int h2 = 0; h2 < 2; ++h2) {
-          uint32_t pk[32];
+        for (int q = 0; q < kBN / 32; ++q) {
+          uint32_t pk[16];
 #pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            const float p0 = ex2(fmaf(__uint_as_float(sr[64 * h2 + 2 * c]), sl2, neg_m));
-            const float p1 = ex2(fmaf(__uint_as_float(sr[64 * h2 + 2 * c + 1]), sl2, neg_m));
-            rs0 += p0;
-            rs1 += p1;
-            pk[c] = pack_bf16x2(p0, p1);
+          for (int i = 0; i < 16; ++i) {
+            const int c = q * 32 + 2 * i;
+            const float2 x = ffma2(make_float2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sl2v, negmv);
+            float2 p;
+            if (kPolyEvery > 0 && (i % kPolyEvery) == kPolyEvery - 1) {
+              p = exp2_poly2(x);
+            } else {
+              p.x = ex2(x.x);
+              p.y = ex2(x.y);
+            }
+            rs = fadd2(rs, p);
+            pk[i] = pack_bf16x2(p.x, p.y);
           }
-          tmem_st32(tS + 32 * h2, pk);
+          tmem_st16(tS + 16 * q, pk);
         }
-        l += rs0 + rs1;
+        l += rs.x + rs.y;
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&bars->p_full[t]);
@@ -288,46 +322,61 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t sQ = smem_u32(smem + C::kOffQ);
         const uint32_t sK = smem_u32(smem + C::kOffK);
         const uint32_t sV = smem_u32(smem + C::kOffV);
-        bool ok = wait_bar(&bars->q_full, 0, w, 3);
+        // S_t = Q_t K^T for key tile j (K from ring stage s)
+        auto issue_s = [&](int t, int s) {
+          const uint32_t qa = sQ + t * C::kTileBytes;
+          const uint32_t kb = sK + s * C::kTileBytes;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * C::kSubBytes + (kk & 3) * 32;
+            umma_ss(tmem + C::colS(t), sw128_desc(qa + off, 16, 1024), sw128_desc(kb + off, 16, 1024),
+                    C::kIdescS, kk > 0 ? 1u : 0u);
+          }
+          umma_commit(&bars->s_full[t]);
+        };
+        // O_t += P_t V_j (P_t from TMEM over S_t, V from ring stage s)
+        auto issue_pv = [&](int t, int s, bool acc) {
+          const uint32_t vb = sV + s * C::kTileBytes;
+#pragma unroll
+          for (int kk = 0; kk < kBN / 16; ++kk) {
+            umma_ts(tmem + C::colO(t), tmem + C::colS(t) + kk * 8, sw128_desc(vb + kk * 2048, C::kSubBytes, 1024),
+                    C::kIdescPV, (acc || kk > 0) ? 1u : 0u);
+          }
+          umma_commit(&bars->o_done[t]);
+        };
+        // Issue order: S_0(0) S_1(0) | PV_0(j) S_0(j+1) PV_1(j) S_1(j+1) | ...
+        // S_t(j+1) overwrites the columns PV_t(j) reads P_t(j) from; the tensor
+        // pipe executes one thread's MMAs in issue order, so PV_t(j) has read
+        // P_t(j) before S_t(j+1) writes there.
+        bool ok = wait_bar(&bars->q_full, 0, w, 3) && wait_bar(&bars->k_full[0], 0, w, 4);
+        if (ok) {
+          tc_fence_after();
+          for (int t = 0; t < 2; ++t)
+            if (nkt[t] > 0) issue_s(t, 0);
+          umma_commit(&bars->k_empty[0]);
+        }
         for (int j = 0; ok && j < nk; ++j) {
           const int s = j % C::kStages;
-          const uint32_t ph = (j / C::kStages) & 1;
-          if (!(ok = wait_bar(&bars->k_full[s], ph, w, 4))) break;
-          tc_fence_after();
-          for (int t = 0; t < 2; ++t) {
-            if (j >= nkt[t]) continue;
-            // S_t is overwritten: the previous P_t must have been consumed.
-            if (j > 0 && !(ok = wait_bar(&bars->o_done[t], (j - 1) & 1, w, 5))) break;
-            tc_fence_after();
-            const uint32_t qa = sQ + t * C::kTileBytes;
-            const uint32_t kb = sK + s * C::kTileBytes;
-#pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-              const uint32_t off = (kk >> 2) * C::kSubBytes + (kk & 3) * 32;
-              umma_ss(tmem + C::colS(t), sw128_desc(qa + off, 16, 1024), sw128_desc(kb + off, 16, 1024),
-                      C::kIdescS, kk > 0 ? 1u : 0u);
-            }
-            umma_commit(&bars->s_full[t]);
-          }
-          if (!ok) break;
-          umma_commit(&bars->k_empty[s]);
-          if (!(ok = wait_bar(&bars->v_full[s], ph, w, 6))) break;
-          tc_fence_after();
+          const int sn = (j + 1) % C::kStages;
+          if (!(ok = wait_bar(&bars->v_full[s], (j / C::kStages) & 1, w, 6))) break;
+          bool next_k = false;
           for (int t = 0; t < 2; ++t) {
             if (j >= nkt[t]) continue;
             if (!(ok = wait_bar(&bars->p_full[t], j & 1, w, 7))) break;
             tc_fence_after();
-            const uint32_t vb = sV + s * C::kTileBytes;
-#pragma unroll
-            for (int kk = 0; kk < kBN / 16; ++kk) {
-              umma_ts(tmem + C::colO(t), tmem + C::colS(t) + kk * 8,
-                      sw128_desc(vb + kk * 2048, C::kSubBytes, 1024), C::kIdescPV,
-                      (j > 0 || kk > 0) ? 1u : 0u);
+            issue_pv(t, s, j > 0);
+            if (j + 1 < nkt[t]) {
+              if (!next_k) {
+                if (!(ok = wait_bar(&bars->k_full[sn], ((j + 1) / C::kStages) & 1, w, 5))) break;
+                tc_fence_after();
+                next_k = true;
+              }
+              issue_s(t, sn);
             }
-            umma_commit(&bars->o_done[t]);
           }
           if (!ok) break;
           umma_commit(&bars->v_empty[s]);
+          if (next_k) umma_commit(&bars->k_empty[sn]);
         }
         // all MMAs of this CTA finish before TMEM is released
         umma_commit(&bars->drain);

@@ -1,0 +1,74 @@
+"""The multi-GPU bench path, exercised with world_size-2 gloo ranks on CPU.
+
+Each GPU runs its own copy of the workload (the heads of attention are
+independent, so nothing crosses between GPUs on the data path).  What the
+ranks share is bookkeeping: every rank draws its own seeded inputs of the same
+shape, the timing is the slowest rank's, and the reported throughput is all
+ranks' FLOPs over that time.
+"""
+
+from __future__ import annotations
+
+import os
+import subprocess
+import sys
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    sys.path.insert(0, ROOT)
+    import bench
+    from exact_io_aware_51_b200 import inputs as I
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        # per-rank inputs: same shape, different seed
+        qi, ki, vi, doi = I.make_inputs(1, 64, 2, 64, seed=rank)
+        shapes = dist_gather_obj((tuple(qi.shape), float(qi.float().sum())), world)
+        # the slowest rank's time is everybody's time
+        local_ms = 10.0 + 5.0 * rank
+        slow = bench.max_over_ranks(local_ms, dist, torch.device("cpu"))
+        value = bench.aggregate_tflops(3.5e12, steps=4, world=world, ms_max=slow)
+        q.put((rank, shapes, slow, value))
+    finally:
+        dist.destroy_process_group()
+
+
+def dist_gather_obj(obj, world):
+    out = [None] * world
+    dist.all_gather_object(out, obj)
+    return out
+
+
+def test_two_ranks_take_the_slowest_time_and_sum_the_work():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = 29500 + (os.getpid() % 1000)
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = [q.get(timeout=120) for _ in procs]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    res.sort()
+    for rank, shapes, slow, value in res:
+        assert slow == 15.0
+        # 2 ranks x 4 steps x 3.5 TFLOP over 15 ms
+        assert value == pytest.approx(2 * 4 * 3.5 / 15e-3)
+        assert shapes[0][0] == shapes[1][0]          # same shape on every rank
+        assert shapes[0][1] != shapes[1][1]          # but each rank's own inputs
+
+
+def test_reference_arm_on_a_non_zero_rank_exits_quietly():
+    env = dict(os.environ, RANK="1", LOCAL_RANK="1", WORLD_SIZE="2", MASTER_ADDR="127.0.0.1")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--gpus", "2",
+                        "--steps", "1", "--warmup", "0"], capture_output=True, text=True, env=env, timeout=300)
+    assert r.returncode == 0, r.stderr
+    assert r.stdout.strip() == ""
