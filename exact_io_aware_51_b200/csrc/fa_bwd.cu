@@ -101,9 +101,14 @@ constexpr int kBN = 128;       // keys per CTA (TMEM lanes of S^T, dP^T, dK, dV)
 constexpr int kBMq = 64;       // query rows per streamed tile
 constexpr int kThreads = 384;  // WG0 P/dS, WG1 dQ drain, WG2 loader + MMA
 constexpr int kStages = 2;
-constexpr uint32_t kRegCompute = 216;  // 384 x 168 = 128 x 216 + 128 x 216 + 128 x 72
+// 384 x 168 at launch = 128 x 216 + 128 x 216 + 128 x 72.  A warpgroup above the
+// launch count raises its share (setmaxnreg.inc), one below lowers it
+// (setmaxnreg.dec); the other direction is an illegal instruction.
+constexpr uint32_t kRegCompute = 216;
 constexpr uint32_t kRegDq = 216;
 constexpr uint32_t kRegOther = 72;
+static_assert(kRegCompute >= 168 && kRegDq >= 168 && kRegOther <= 168, "setmaxnreg direction");
+static_assert(kRegCompute + kRegDq + kRegOther == 3 * 168, "register split must match the launch");
 
 struct BwdCfg {
   static constexpr int D = 128;

@@ -41,6 +41,8 @@ constexpr int kThreads = 384;   // WG0, WG1: softmax; WG2: loader warp, MMA warp
 // Register split (per thread): 384 x 168 at launch = 256 x 216 + 128 x 72.
 constexpr uint32_t kRegSoftmax = 216;
 constexpr uint32_t kRegOther = 72;
+static_assert(kRegSoftmax >= 168 && kRegOther <= 168, "setmaxnreg direction (launch count 168)");
+static_assert(2 * kRegSoftmax + kRegOther == 3 * 168, "register split must match the launch");
 constexpr float kTau = 8.0f;    // lazy-rescale threshold (log2 units)
 // When > 0, one score pair in kPolyEvery takes its exponentials on the FMA pipe
 // (exp2_poly2) instead of the MUFU unit.  Measured on B200 at d = 128 the MUFU
@@ -235,8 +237,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int i = 0; i < 16; ++i) {
             const int c = q * 32 + 2 * i;
             const float2 x = ffma2(make_float2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sl2v, negmv);
-            float2 p;
-            if (kPolyEvery > 0 && (i % kPolyEvery) == kPolyEvery - 1) {
+            float2 p = make_float2(0.f, 0.f);
+            bool poly = false;
+            if constexpr (kPolyEvery > 0) poly = (i % (kPolyEvery > 0 ? kPolyEvery : 1)) == kPolyEvery - 1;
+            if (poly) {
               p = exp2_poly2(x);
             } else {
               p.x = ex2(x.x);
