@@ -33,7 +33,7 @@ _LIB = None
 # Every symbol include/fa.h declares.
 EXPORTED = ("fa_fwd", "fa_bwd_workspace_size", "fa_bwd", "fa_status_string", "fa_last_cuda_error",
             "fa_last_device_status", "fa_set_wait_limit_ms", "fa_debug_inject", "fa_debug_umma",
-            "fa_version", "fa_set_kernel_events")
+            "fa_version", "fa_set_kernel_events", "fa_bwd_static_scratch")
 
 
 class FAError(RuntimeError):
@@ -79,6 +79,8 @@ def lib() -> ctypes.CDLL:
     L.fa_debug_inject.restype = None
     L.fa_debug_umma.argtypes = [vp, vp, vp, i, i, i, i, i, vp]
     L.fa_debug_umma.restype = i
+    L.fa_bwd_static_scratch.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, i, vp]
+    L.fa_bwd_static_scratch.restype = i
     L.fa_set_kernel_events.argtypes = [vp, vp]
     L.fa_set_kernel_events.restype = None
     L.fa_version.argtypes = []

@@ -109,6 +109,28 @@ int fa_bwd(const void* Q, const void* K, const void* V, const void* O, const voi
            void* dK, void* dV, int B, int H, int N, int d, float scale, int causal, int dtype, void* workspace,
            size_t workspace_bytes, void* stream);
 
+/*
+ * fa_bwd for callers that cannot allocate device memory when they run the
+ * backward pass (runtimes whose device memory is laid out once at start-up,
+ * or code that must not call cudaMalloc mid-run because it can synchronise
+ * the device or fail under memory pressure).  The pages have no counterpart
+ * to this entry point; it is a service of this library.
+ *   Same arguments and results as fa_bwd, minus the workspace: the scratch is
+ *   a 64 MiB array compiled into the library, which every GPU that loads the
+ *   library holds until the process exits.  The call allocates nothing.
+ *   A problem whose fa_bwd_workspace_size() exceeds 64 MiB is refused with
+ *   FA_ERR_TOO_LARGE.
+ *   All calls share that one array.  Each call's first kernel rewrites what
+ *   the later ones read, so results never depend on an earlier call, but
+ *   calls whose kernels overlap on the GPU (other streams, or other host
+ *   threads without ordering) race on it and give wrong gradients.
+ *   The first call on a device looks up the array's device address with that
+ *   device current; make it before any stream capture.
+ */
+int fa_bwd_static_scratch(const void* Q, const void* K, const void* V, const void* O, const void* dO,
+                          const float* LSE, void* dQ, void* dK, void* dV, int B, int H, int N, int d, float scale,
+                          int causal, int dtype, void* stream);
+
 /* Static English text for a status code. */
 const char* fa_status_string(int status);
 
