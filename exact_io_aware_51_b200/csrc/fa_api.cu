@@ -144,7 +144,9 @@ int check_scale(float scale) {
 
 }  // namespace
 
-CUresult make_tile_map(CUtensorMap* map, const void* base, int B, int N, int H, int d, int rows) {
+namespace {
+// The driver's TMA descriptor encoder, looked up once through the runtime.
+PFN_cuTensorMapEncodeTiled_v12000 encoder() {
   std::call_once(g_encode_once, [] {
     void* fn = nullptr;
     cudaDriverEntryPointQueryResult q;
@@ -152,7 +154,12 @@ CUresult make_tile_map(CUtensorMap* map, const void* base, int B, int N, int H, 
         q == cudaDriverEntryPointSuccess)
       g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
   });
-  if (!g_encode) return CUDA_ERROR_NOT_FOUND;
+  return g_encode;
+}
+}  // namespace
+
+CUresult make_tile_map(CUtensorMap* map, const void* base, int B, int N, int H, int d, int rows) {
+  if (!encoder()) return CUDA_ERROR_NOT_FOUND;
   // dims innermost first: feature, sequence, head, batch
   const cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(H),
                               static_cast<cuuint64_t>(B)};
@@ -163,6 +170,18 @@ CUresult make_tile_map(CUtensorMap* map, const void* base, int B, int N, int H, 
   return g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+}
+
+CUresult make_dq_accum_map(CUtensorMap* map, float* base, int B, int N, int H, int d) {
+  if (!encoder()) return CUDA_ERROR_NOT_FOUND;
+  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(H),
+                              static_cast<cuuint64_t>(B)};
+  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(H) * d * 4, static_cast<cuuint64_t>(d) * 4,
+                                 static_cast<cuuint64_t>(N) * H * d * 4};
+  const cuuint32_t box[4] = {static_cast<cuuint32_t>(d), 64u, 1u, 1u};
+  const cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+  return g_encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
 }
 
 }  // namespace fa
@@ -306,17 +325,18 @@ int fa_bwd(const void* Q, const void* K, const void* V, const void* O, const voi
   ws += align256(static_cast<size_t>(B) * H * npad * sizeof(float));
   a.LSE2 = reinterpret_cast<float*>(ws);
 
-  CUtensorMap tq, tk, tv, tdo;
+  CUtensorMap tq, tk, tv, tdo, tdq;
   CUresult r;
-  if ((r = make_tile_map(&tq, Q, B, N, H, d, 64)) != CUDA_SUCCESS ||
-      (r = make_tile_map(&tdo, dO, B, N, H, d, 64)) != CUDA_SUCCESS ||
+  if ((r = make_tile_map(&tq, Q, B, N, H, d, 128)) != CUDA_SUCCESS ||
+      (r = make_tile_map(&tdo, dO, B, N, H, d, 128)) != CUDA_SUCCESS ||
       (r = make_tile_map(&tk, K, B, N, H, d, 128)) != CUDA_SUCCESS ||
-      (r = make_tile_map(&tv, V, B, N, H, d, 128)) != CUDA_SUCCESS)
+      (r = make_tile_map(&tv, V, B, N, H, d, 128)) != CUDA_SUCCESS ||
+      (r = make_dq_accum_map(&tdq, a.dQacc, B, N, H, d)) != CUDA_SUCCESS)
     return fail_encode(r);
   cudaError_t e = launch_bwd_pre(a, s);
   if (e != cudaSuccess) return fail_cuda(e);
   if (t_ev_start) cudaEventRecord(t_ev_start, s);
-  e = launch_bwd_main(tq, tk, tv, tdo, a, make_ctl(*st), s);
+  e = launch_bwd_main(tq, tk, tv, tdo, tdq, a, make_ctl(*st), s);
   if (e != cudaSuccess) return fail_cuda(e);
   if (t_ev_stop) cudaEventRecord(t_ev_stop, s);
   e = launch_bwd_dq(a, s);

@@ -97,53 +97,58 @@ __global__ void __launch_bounds__(256) bwd_dq_kernel(const BwdArgs a, long long 
 // ---------------------------------------------------------------------------
 // 2. main kernel (D = 128)
 // ---------------------------------------------------------------------------
-constexpr int kBN = 128;       // keys per CTA (TMEM lanes of S^T, dP^T, dK, dV)
-constexpr int kBMq = 64;       // query rows per streamed tile
-constexpr int kThreads = 384;  // WG0 P/dS, WG1 dQ drain, WG2 loader + MMA
-constexpr int kStages = 2;
-// 384 x 168 at launch = 128 x 216 + 128 x 216 + 128 x 72.  A warpgroup above the
+constexpr int kBN = 128;        // keys per CTA (TMEM lanes of S^T, dP^T, dK, dV)
+constexpr int kBMq = 128;       // query rows per streamed tile
+constexpr int kThreads = 512;   // WG0, WG1: P / dS for query columns 0-63 / 64-127; WG2: dQ drain; WG3: loader + MMA
+constexpr int kStages = 2;      // Q/dO ring
+// 512 x 128 at launch = 2 x 128 x 168 + 128 x 104 + 128 x 72.  A warpgroup above the
 // launch count raises its share (setmaxnreg.inc), one below lowers it
 // (setmaxnreg.dec); the other direction is an illegal instruction.
-constexpr uint32_t kRegCompute = 216;
-constexpr uint32_t kRegDq = 216;
-constexpr uint32_t kRegOther = 72;
-static_assert(kRegCompute >= 168 && kRegDq >= 168 && kRegOther <= 168, "setmaxnreg direction");
-static_assert(kRegCompute + kRegDq + kRegOther == 3 * 168, "register split must match the launch");
+constexpr uint32_t kRegLaunch = 128;
+constexpr uint32_t kRegCompute = 168;
+constexpr uint32_t kRegDrain = 104;
+constexpr uint32_t kRegCtrl = 72;
+static_assert(kRegCompute >= kRegLaunch && kRegDrain <= kRegLaunch && kRegCtrl <= kRegLaunch,
+              "setmaxnreg direction");
+static_assert(2 * kRegCompute + kRegDrain + kRegCtrl == 4 * kRegLaunch, "register split must match the launch");
 
 struct BwdCfg {
   static constexpr int D = 128;
-  static constexpr int kKVBytes = kBN * D * 2;    // 32 KB: two [128][64] sub-tiles
-  static constexpr int kKVSub = kBN * 128;        // 16 KB
-  static constexpr int kQBytes = kBMq * D * 2;    // 16 KB: two [64][64] sub-tiles
-  static constexpr int kQSub = kBMq * 128;        // 8 KB
-  static constexpr int kPBytes = kBN * kBMq * 2;  // 16 KB: one [128][64] tile
+  static constexpr int kSub = kBN * 128;          // one [128 rows][64] bf16 SW128 sub-tile: 16 KB
+  static constexpr int kTile = 2 * kSub;          // one 128 x 128 bf16 tile: 32 KB
   static constexpr int kOffK = 0;
-  static constexpr int kOffV = kOffK + kKVBytes;
-  static constexpr int kOffQ = kOffV + kKVBytes;
-  static constexpr int kOffDO = kOffQ + kStages * kQBytes;
-  static constexpr int kOffPt = kOffDO + kStages * kQBytes;
-  static constexpr int kOffDSt = kOffPt + kPBytes;
-  static constexpr int kOffL = kOffDSt + kPBytes;       // [stage][64] fp32 LSE2
-  static constexpr int kOffDv = kOffL + kStages * 256;  // [stage][64] fp32 D
-  static constexpr int kOffBar = kOffDv + kStages * 256;
-  static constexpr int kSmemBytes = kOffBar + 512 + 1024;
-  // TMEM columns
-  static constexpr uint32_t kColDV = 0, kColDK = 128, kColS = 256, kColDP = 320, kColDQ = 384;
-  static constexpr uint32_t kIdescS = idesc_bf16(kBN, kBMq, 0, 0);   // S^T, dP^T
-  static constexpr uint32_t kIdescKV = idesc_bf16(kBN, D, 0, 1);     // dV, dK
-  static constexpr uint32_t kIdescQ = idesc_bf16(D, kBMq, 1, 1);     // dQ^T
+  static constexpr int kOffV = kOffK + kTile;
+  static constexpr int kOffQ = kOffV + kTile;                 // [stage] Q_i
+  static constexpr int kOffDO = kOffQ + kStages * kTile;      // [stage] dO_i, then dS^T_i
+  static constexpr int kOffL = kOffDO + kStages * kTile;      // [stage][128] fp32 LSE * log2 e
+  static constexpr int kOffDv = kOffL + kStages * 512;        // [stage][128] fp32 rowsum(dO * O)
+  static constexpr int kOffDQS = kOffDv + kStages * 512;       // [64 q][128 d] fp32 dQ staging
+  static constexpr int kOffBar = kOffDQS + 64 * 128 * 4;
+  // no alignment slack: the dynamic shared memory is declared 1024-aligned and checked
+  static constexpr int kSmemBytes = kOffBar + 256;
+  // TMEM columns: dV | dK | R1 | R2.
+  //   R1: S^T_i (fp32), then P^T_i as bf16 pairs in columns [0, 32) (query
+  //       columns 0-63) and [64, 96) (query columns 64-127).
+  //   R2: dP^T_i (fp32), then dS^T_i as bf16 pairs at the same places, then
+  //       dQ_i^T (fp32, features on lanes) once dK_i has read dS^T_i.
+  static constexpr uint32_t kColDV = 0, kColDK = 128, kColR1 = 256, kColR2 = 384;
+  static constexpr uint32_t kIdescS = idesc_bf16(kBN, kBMq, 0, 0);   // S^T, dP^T: K-major A and B
+  static constexpr uint32_t kIdescKV = idesc_bf16(kBN, D, 0, 1);     // dV, dK: A from TMEM, B MN-major
+  static constexpr uint32_t kIdescQ = idesc_bf16(D, kBMq, 1, 1);     // dQ^T: both MN-major
 };
 
 struct BwdBars {
   uint64_t kv_full;
   uint64_t q_full[kStages], q_empty[kStages];
-  uint64_t s_full, dp_full, pt_ready, ds_ready;
-  uint64_t dq_full[2], dq_free[2];
+  uint64_t s_full, dp_full, pt_ready, ds_ready, dv_done, dq_full, dq_free;
   uint64_t acc_done;
   uint64_t drain;
+  uint64_t stage_sync;  // the dQ drain warpgroup's internal barrier
   uint32_t tmem_base;
   int abort;
 };
+static_assert(sizeof(BwdBars) <= 256, "barrier block");
+static_assert(BwdCfg::kOffDQS % 1024 == 0 && BwdCfg::kSmemBytes <= 232448, "shared memory layout");
 
 __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, unsigned long long limit_ns) {
   const uint64_t t0 = globaltimer_ns();
@@ -154,28 +159,36 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, unsig
 
 __device__ __forceinline__ bool warp_all(bool ok) { return __all_sync(0xffffffffu, ok); }
 
-__device__ __forceinline__ void red_add_f32(float* p, float v) {
-  asm volatile("red.global.add.f32 [%0], %1;" ::"l"(p), "f"(v) : "memory");
+// TMA reduce-add of a shared-memory tile into global memory (fp32), and the
+// bulk-group bookkeeping around it.
+__device__ __forceinline__ void tma_reduce_add_4d(const CUtensorMap* map, const void* src, int c0, int c1, int c2,
+                                                  int c3) {
+  asm volatile(
+      "cp.reduce.async.bulk.tensor.4d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::"l"(
+          reinterpret_cast<uint64_t>(map)),
+      "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+      : "memory");
 }
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
-// write one 64-value bf16 row (row r of a [128][64] SW128 tile)
-__device__ __forceinline__ void store_row_sw128(uint32_t tile, int r, const float* v) {
-#pragma unroll
-  for (int u = 0; u < 8; ++u) {
-    st_shared_v4(tile + sw128_offset(r, u), pack_bf16x2(v[8 * u + 0], v[8 * u + 1]),
-                 pack_bf16x2(v[8 * u + 2], v[8 * u + 3]), pack_bf16x2(v[8 * u + 4], v[8 * u + 5]),
-                 pack_bf16x2(v[8 * u + 6], v[8 * u + 7]));
-  }
-}
+// TMEM column of the bf16 pairs for reduction step kk (16 query columns) of a
+// P^T / dS^T tile written by the two compute warpgroups.
+__device__ __forceinline__ uint32_t ts_col(int kk) { return (kk < 4) ? kk * 8 : 64 + (kk - 4) * 8; }
 
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
-                    const BwdArgs a, const DevCtl ctl) {
+                    const __grid_constant__ CUtensorMap tmDQ, const BwdArgs a, const DevCtl ctl) {
   using C = BwdCfg;
   constexpr int D = C::D;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = smem_raw;
+  if (smem_u32(smem) & 1023u) {  // the swizzled layouts need a 1024-byte aligned base
+    if (threadIdx.x == 0) atomicCAS(ctl.status, 0, kDevTimeout | 0xA1);
+    return;
+  }
   BwdBars* bars = reinterpret_cast<BwdBars*>(smem + C::kOffBar);
   const int warp = warp_id();
   const int lane = lane_id();
@@ -185,8 +198,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int b = blockIdx.z;
   const int key0 = jt * kBN;
   const int nq_total = (a.N + kBMq - 1) / kBMq;
-  const int i0 = a.causal ? (key0 / kBMq) : 0;  // first query tile that sees these keys
+  const int i0 = a.causal ? jt : 0;  // first query tile that sees these keys
   const int nq = max(0, nq_total - i0);
+  auto qtile = [&](int i) { return i0 + i; };
   const size_t bh = static_cast<size_t>(b) * a.H + h;
 
   if (threadIdx.x == 0) {
@@ -197,242 +211,296 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(&bars->s_full, 1);
     mbar_init(&bars->dp_full, 1);
-    mbar_init(&bars->pt_ready, 128);
-    mbar_init(&bars->ds_ready, 128);
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&bars->dq_full[s], 1);
-      mbar_init(&bars->dq_free[s], 128);
-    }
+    mbar_init(&bars->pt_ready, 256);
+    mbar_init(&bars->ds_ready, 256);
+    mbar_init(&bars->dv_done, 1);
+    mbar_init(&bars->dq_full, 1);
+    mbar_init(&bars->dq_free, 128);
     mbar_init(&bars->acc_done, 1);
     mbar_init(&bars->drain, 1);
+    mbar_init(&bars->stage_sync, 128);
     bars->abort = (*reinterpret_cast<volatile unsigned int*>(ctl.abort_epoch) == ctl.epoch) ? 1 : 0;
     fence_mbar_init();
   }
-  if (warp == 9) tmem_alloc(&bars->tmem_base, 512);
+  if (warp == 13) tmem_alloc(&bars->tmem_base, 512);
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
   const WaitCtl w{&bars->abort, ctl.status, ctl.abort_epoch, ctl.epoch, ctl.limit_ns};
 
-  if (warp < 4) {
-    // ===================== P^T / dS^T warpgroup =====================
+  if (warp < 8) {
+    // ===================== P^T / dS^T warpgroups =====================
+    // WG g owns query columns [64 g, 64 g + 64) of every tile.
     reg_alloc<kRegCompute>();
     if (bars->abort == 0) {
-      const int r = warp * 32 + lane;  // key row within the tile = TMEM lane
+      const int g = warp >> 2;
+      const int quarter = warp & 3;
+      const int r = quarter * 32 + lane;  // key row within the tile = TMEM lane
       const int key = key0 + r;
-      const uint32_t lane_bits = static_cast<uint32_t>(warp * 32) << 16;
-      const uint32_t sPt = smem_u32(smem + C::kOffPt);
-      const uint32_t sDSt = smem_u32(smem + C::kOffDSt);
+      const uint32_t lane_bits = static_cast<uint32_t>(quarter * 32) << 16;
+      const uint32_t tR1 = tmem + lane_bits + C::kColR1 + 64 * g;  // this WG's 64 fp32 columns
+      const uint32_t tR2 = tmem + lane_bits + C::kColR2 + 64 * g;
       const float sl2 = a.scale_log2;
       bool ok = true;
-      for (int it = 0; it < nq; ++it) {
-        const int st = it % kStages;
-        const int q0 = (i0 + it) * kBMq;
-        ok = warp_all(wait_bar(&bars->q_full[st], (it / kStages) & 1, w, 20));
+      for (int i = 0; i < nq; ++i) {
+        const int st = i % kStages;
+        const uint32_t par = i & 1;
+        const int q0 = qtile(i) * kBMq + 64 * g;  // first query column of this WG
+        ok = warp_all(wait_bar(&bars->q_full[st], (i / kStages) & 1, w, 20));
         if (!ok) break;
-        ok = warp_all(wait_bar(&bars->s_full, it & 1, w, 21));
+        ok = warp_all(wait_bar(&bars->s_full, par, w, 21));
         if (!ok) break;
         tc_fence_after();
-        uint32_t sr[kBMq];
-        tmem_ld32(tmem + lane_bits + C::kColS, sr);
-        tmem_ld32(tmem + lane_bits + C::kColS + 32, sr + 32);
+        uint32_t sr[64];
+        tmem_ld32(tR1, sr);
+        tmem_ld32(tR1 + 32, sr + 32);
         tmem_wait_ld();
         reg_fence32(sr);
         reg_fence32(sr + 32);
-        const float* sL = reinterpret_cast<const float*>(smem + C::kOffL + st * 256);
-        const float* sD = reinterpret_cast<const float*>(smem + C::kOffDv + st * 256);
-        float p[kBMq];
-        const bool need_mask = (q0 + kBMq > a.N) || (key0 + kBN > a.N) || (a.causal && q0 < key0 + kBN);
+        const float4* sL = reinterpret_cast<const float4*>(smem + C::kOffL + st * 512 + 256 * g);
+        const float4* sD = reinterpret_cast<const float4*>(smem + C::kOffDv + st * 512 + 256 * g);
+        float p[64];
 #pragma unroll
-        for (int c = 0; c < kBMq; ++c) p[c] = ex2(fmaf(__uint_as_float(sr[c]), sl2, -sL[c]));
+        for (int c4 = 0; c4 < 16; ++c4) {
+          const float4 l4 = sL[c4];
+          const float2 x0 = ffma2(make_float2(__uint_as_float(sr[4 * c4]), __uint_as_float(sr[4 * c4 + 1])),
+                                  make_float2(sl2, sl2), make_float2(-l4.x, -l4.y));
+          const float2 x1 = ffma2(make_float2(__uint_as_float(sr[4 * c4 + 2]), __uint_as_float(sr[4 * c4 + 3])),
+                                  make_float2(sl2, sl2), make_float2(-l4.z, -l4.w));
+          p[4 * c4 + 0] = ex2(x0.x);
+          p[4 * c4 + 1] = ex2(x0.y);
+          p[4 * c4 + 2] = ex2(x1.x);
+          p[4 * c4 + 3] = ex2(x1.y);
+        }
+        const bool need_mask = (q0 + 64 > a.N) || (key0 + kBN > a.N) || (a.causal && q0 < key0 + kBN);
         if (need_mask) {
 #pragma unroll
-          for (int c = 0; c < kBMq; ++c) {
+          for (int c = 0; c < 64; ++c) {
             const int q = q0 + c;
             const bool vis = (q < a.N) && (key < a.N) && (!a.causal || q >= key);
             if (!vis) p[c] = 0.f;
           }
         }
-        store_row_sw128(sPt, r, p);
-        fence_proxy_async_smem();
+        {  // P^T (bf16 pairs) over the first 32 of this WG's R1 columns
+          uint32_t pk[32];
+#pragma unroll
+          for (int c = 0; c < 32; ++c) pk[c] = pack_bf16x2(p[2 * c], p[2 * c + 1]);
+          tmem_st32(tR1, pk);
+          tmem_wait_st();
+        }
         tc_fence_before();
         mbar_arrive(&bars->pt_ready);
 
-        ok = warp_all(wait_bar(&bars->dp_full, it & 1, w, 22));
+        ok = warp_all(wait_bar(&bars->dp_full, par, w, 22));
         if (!ok) break;
         tc_fence_after();
-        uint32_t dr[kBMq];
-        tmem_ld32(tmem + lane_bits + C::kColDP, dr);
-        tmem_ld32(tmem + lane_bits + C::kColDP + 32, dr + 32);
+        uint32_t dr[64];
+        tmem_ld32(tR2, dr);
+        tmem_ld32(tR2 + 32, dr + 32);
         tmem_wait_ld();
         reg_fence32(dr);
         reg_fence32(dr + 32);
+        uint32_t pk[32];
 #pragma unroll
-        for (int c = 0; c < kBMq; ++c) p[c] = p[c] * (__uint_as_float(dr[c]) - sD[c]);
-        store_row_sw128(sDSt, r, p);
+        for (int c4 = 0; c4 < 16; ++c4) {
+          const float4 d4 = sD[c4];
+          pk[2 * c4] = pack_bf16x2(p[4 * c4 + 0] * (__uint_as_float(dr[4 * c4 + 0]) - d4.x),
+                                   p[4 * c4 + 1] * (__uint_as_float(dr[4 * c4 + 1]) - d4.y));
+          pk[2 * c4 + 1] = pack_bf16x2(p[4 * c4 + 2] * (__uint_as_float(dr[4 * c4 + 2]) - d4.z),
+                                       p[4 * c4 + 3] * (__uint_as_float(dr[4 * c4 + 3]) - d4.w));
+        }
+        // dS^T into TMEM (A operand of dK) ...
+        tmem_st32(tR2, pk);
+        // ... and into shared memory over dO_i (B operand of dQ^T) once dV_i has read dO_i
+        ok = warp_all(wait_bar(&bars->dv_done, par, w, 24));
+        if (!ok) break;
+        const uint32_t sDSt = smem_u32(smem + C::kOffDO + st * C::kTile + g * C::kSub);
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          st_shared_v4(sDSt + sw128_offset(r, u), pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
         fence_proxy_async_smem();
+        tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&bars->ds_ready);
       }
-      // ---- epilogue: dV and dK rows of this key ----
+      // ---- epilogue: WG0 writes the dV rows, WG1 the dK rows of its keys ----
+      if (ok && nq > 0) ok = warp_all(wait_bar(&bars->acc_done, 0, w, 23));
       if (ok) {
-        if (nq > 0) ok = warp_all(wait_bar(&bars->acc_done, 0, w, 23));
-        if (ok) {
-          tc_fence_after();
-          const size_t base = ((static_cast<size_t>(b) * a.N + key) * a.H + h) * D;
-          __nv_bfloat16* dv = reinterpret_cast<__nv_bfloat16*>(a.dV) + base;
-          __nv_bfloat16* dk = reinterpret_cast<__nv_bfloat16*>(a.dK) + base;
+        tc_fence_after();
+        const size_t base = ((static_cast<size_t>(b) * a.N + key) * a.H + h) * D;
+        const uint32_t col = g == 0 ? C::kColDV : C::kColDK;
+        const float mul = g == 0 ? 1.f : a.scale;
+        __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(g == 0 ? a.dV : a.dK) + base;
 #pragma unroll
-          for (int which = 0; which < 2; ++which) {
-            const uint32_t col = which == 0 ? C::kColDV : C::kColDK;
-            const float mul = which == 0 ? 1.f : a.scale;
-            __nv_bfloat16* dst = which == 0 ? dv : dk;
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t v[32];
+          if (nq > 0) {
+            tmem_ld32(tmem + lane_bits + col + c * 32, v);
+            tmem_wait_ld();
+            reg_fence32(v);
+          } else {
 #pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
-              uint32_t v[32];
-              if (nq > 0) {
-                tmem_ld32(tmem + lane_bits + col + c * 32, v);
-                tmem_wait_ld();
-                reg_fence32(v);
-              } else {
+            for (int i = 0; i < 32; ++i) v[i] = 0u;
+          }
+          uint32_t pk[16];
 #pragma unroll
-                for (int i = 0; i < 32; ++i) v[i] = 0u;
-              }
-              uint32_t pk[16];
+          for (int i = 0; i < 16; ++i)
+            pk[i] = pack_bf16x2(__uint_as_float(v[2 * i]) * mul, __uint_as_float(v[2 * i + 1]) * mul);
+          if (key < a.N) {
 #pragma unroll
-              for (int i = 0; i < 16; ++i)
-                pk[i] = pack_bf16x2(__uint_as_float(v[2 * i]) * mul, __uint_as_float(v[2 * i + 1]) * mul);
-              if (key < a.N) {
-#pragma unroll
-                for (int i = 0; i < 4; ++i)
-                  st_global_v4(dst + c * 32 + i * 8, pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
-              }
-            }
+            for (int i = 0; i < 4; ++i)
+              st_global_v4(dst + c * 32 + i * 8, pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
           }
         }
       }
     }
-  } else if (warp < 8) {
+  } else if (warp < 12) {
     // ===================== dQ drain warpgroup =====================
-    reg_alloc<kRegDq>();
+    // dQ_i^T leaves TMEM as soon as it has been read (so dP_{i+1} can reuse
+    // the columns); each 64-query half is then written to a shared-memory
+    // staging tile [64 q][128 d] and added into the fp32 accumulator in global
+    // memory by one TMA reduce-add (whole lines, no per-element atomics).
+    reg_dealloc<kRegDrain>();
     if (bars->abort == 0) {
       const int quarter = warp & 3;
       const int dd = quarter * 32 + lane;  // feature index = TMEM lane of dQ^T
-      const uint32_t lane_bits = static_cast<uint32_t>(quarter * 32) << 16;
-      for (int it = 0; it < nq; ++it) {
-        const int buf = it & 1;
-        if (!warp_all(wait_bar(&bars->dq_full[buf], (it >> 1) & 1, w, 30))) break;
+      const uint32_t tQ = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + C::kColR2;
+      float* stage = reinterpret_cast<float*>(smem + C::kOffDQS);
+      const bool issuer = (dd == 0);
+      uint32_t sync_phase = 0;
+      bool ok = true;
+      // all 128 drain threads meet here (bounded wait)
+      auto drain_sync = [&]() -> bool {
+        mbar_arrive(&bars->stage_sync);
+        const bool r = warp_all(wait_bar(&bars->stage_sync, sync_phase & 1, w, 31));
+        ++sync_phase;
+        return r;
+      };
+      // write 64 query rows of dQ^T (this thread's feature) into the staging tile and reduce them
+      auto stage_and_reduce = [&](const uint32_t* v, int q_row0) -> bool {
+        if (issuer) bulk_wait_read_all();  // the previous reduction has read the staging tile
+        if (!drain_sync()) return false;
+#pragma unroll
+        for (int c = 0; c < 64; ++c) stage[c * 128 + dd] = __uint_as_float(v[c]);
+        fence_proxy_async_smem();
+        if (!drain_sync()) return false;
+        if (issuer) {
+          tma_reduce_add_4d(&tmDQ, stage, 0, q_row0, h, b);
+          bulk_commit();
+        }
+        return true;
+      };
+      for (int i = 0; ok && i < nq; ++i) {
+        if (!(ok = warp_all(wait_bar(&bars->dq_full, i & 1, w, 30)))) break;
         tc_fence_after();
-        uint32_t v[kBMq];
-        tmem_ld32(tmem + lane_bits + C::kColDQ + buf * 64, v);
-        tmem_ld32(tmem + lane_bits + C::kColDQ + buf * 64 + 32, v + 32);
+        const int q0 = qtile(i) * kBMq;
+        uint32_t v[64];
+        tmem_ld32(tQ, v);
+        tmem_ld32(tQ + 32, v + 32);
+        tmem_wait_ld();
+        reg_fence32(v);
+        reg_fence32(v + 32);
+        if (!(ok = stage_and_reduce(v, q0))) break;
+        tmem_ld32(tQ + 64, v);
+        tmem_ld32(tQ + 96, v + 32);
         tmem_wait_ld();
         reg_fence32(v);
         reg_fence32(v + 32);
         tc_fence_before();
-        mbar_arrive(&bars->dq_free[buf]);
-        const int q0 = (i0 + it) * kBMq;
-        float* dst = a.dQacc + ((static_cast<size_t>(b) * a.N + q0) * a.H + h) * D + dd;
-        const size_t row_stride = static_cast<size_t>(a.H) * D;
-        const int rows = min(kBMq, a.N - q0);
-#pragma unroll
-        for (int c = 0; c < kBMq; ++c)
-          if (c < rows) red_add_f32(dst + c * row_stride, __uint_as_float(v[c]));
+        mbar_arrive(&bars->dq_free);
+        ok = stage_and_reduce(v, q0 + 64);
       }
+      if (issuer) bulk_wait_all();
     }
   } else {
-    reg_dealloc<kRegOther>();
-    if (bars->abort == 0 && warp == 8) {
+    reg_dealloc<kRegCtrl>();
+    if (bars->abort == 0 && warp == 12) {
       // ===================== TMA producer =====================
       if (lane == 0) {
         tma_prefetch_desc(&tmQ);
         tma_prefetch_desc(&tmK);
         tma_prefetch_desc(&tmV);
         tma_prefetch_desc(&tmDO);
-        mbar_arrive_expect_tx(&bars->kv_full, 2 * C::kKVBytes);
+        mbar_arrive_expect_tx(&bars->kv_full, 2 * C::kTile);
         for (int c = 0; c < D / 64; ++c) {
-          tma_load_4d(smem + C::kOffK + c * C::kKVSub, &tmK, &bars->kv_full, c * 64, key0, h, b);
-          tma_load_4d(smem + C::kOffV + c * C::kKVSub, &tmV, &bars->kv_full, c * 64, key0, h, b);
+          tma_load_4d(smem + C::kOffK + c * C::kSub, &tmK, &bars->kv_full, c * 64, key0, h, b);
+          tma_load_4d(smem + C::kOffV + c * C::kSub, &tmV, &bars->kv_full, c * 64, key0, h, b);
         }
-        for (int it = 0; it < nq; ++it) {
-          const int st = it % kStages;
-          const int n = it / kStages;
-          if (it >= kStages && !wait_bar(&bars->q_empty[st], (n - 1) & 1, w, 10)) break;
-          const int q0 = (i0 + it) * kBMq;
-          mbar_arrive_expect_tx(&bars->q_full[st], 2 * C::kQBytes + 512);
+        for (int i = 0; i < nq; ++i) {
+          const int st = i % kStages;
+          const int n = i / kStages;
+          if (i >= kStages && !wait_bar(&bars->q_empty[st], (n - 1) & 1, w, 10)) break;
+          const int q0 = qtile(i) * kBMq;
+          mbar_arrive_expect_tx(&bars->q_full[st], 2 * C::kTile + 1024);
           for (int c = 0; c < D / 64; ++c) {
-            tma_load_4d(smem + C::kOffQ + st * C::kQBytes + c * C::kQSub, &tmQ, &bars->q_full[st], c * 64, q0, h, b);
-            tma_load_4d(smem + C::kOffDO + st * C::kQBytes + c * C::kQSub, &tmDO, &bars->q_full[st], c * 64, q0, h,
-                        b);
+            tma_load_4d(smem + C::kOffQ + st * C::kTile + c * C::kSub, &tmQ, &bars->q_full[st], c * 64, q0, h, b);
+            tma_load_4d(smem + C::kOffDO + st * C::kTile + c * C::kSub, &tmDO, &bars->q_full[st], c * 64, q0, h, b);
           }
-          bulk_load(smem + C::kOffL + st * 256, a.LSE2 + bh * a.Npad + q0, 256, &bars->q_full[st]);
-          bulk_load(smem + C::kOffDv + st * 256, a.Dvec + bh * a.Npad + q0, 256, &bars->q_full[st]);
+          bulk_load(smem + C::kOffL + st * 512, a.LSE2 + bh * a.Npad + q0, 512, &bars->q_full[st]);
+          bulk_load(smem + C::kOffDv + st * 512, a.Dvec + bh * a.Npad + q0, 512, &bars->q_full[st]);
         }
       }
-    } else if (bars->abort == 0 && warp == 9) {
+    } else if (bars->abort == 0 && warp == 13) {
       // ===================== MMA issuer =====================
       if (lane == 0 && nq > 0) {
         const uint32_t sK = smem_u32(smem + C::kOffK);
         const uint32_t sV = smem_u32(smem + C::kOffV);
         const uint32_t sQ = smem_u32(smem + C::kOffQ);
         const uint32_t sDO = smem_u32(smem + C::kOffDO);
-        const uint32_t sPt = smem_u32(smem + C::kOffPt);
-        const uint32_t sDSt = smem_u32(smem + C::kOffDSt);
-        // S^T = K Q^T (or dP^T = V dO^T): A [128 keys][128 d] K-major, B [64 q][128 d] K-major
+        // S^T = K Q^T (or dP^T = V dO^T): A [128 keys][128 d] K-major, B [128 q][128 d] K-major
         auto issue_s = [&](uint32_t a_base, uint32_t b_base, uint32_t col) {
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t ao = (kk >> 2) * C::kKVSub + (kk & 3) * 32;
-            const uint32_t bo = (kk >> 2) * C::kQSub + (kk & 3) * 32;
-            umma_ss(tmem + col, sw128_desc(a_base + ao, 16, 1024), sw128_desc(b_base + bo, 16, 1024), C::kIdescS,
+            const uint32_t off = (kk >> 2) * C::kSub + (kk & 3) * 32;
+            umma_ss(tmem + col, sw128_desc(a_base + off, 16, 1024), sw128_desc(b_base + off, 16, 1024), C::kIdescS,
                     kk > 0 ? 1u : 0u);
           }
         };
-        // dV += P^T dO (or dK += dS^T Q): A [128 keys][64 q] K-major, B [64 q][128 d] MN-major
-        auto issue_kv = [&](uint32_t a_base, uint32_t b_base, uint32_t col, bool acc) {
+        // dV += P^T dO (or dK += dS^T Q): A from TMEM (bf16 pairs), B [128 q][128 d] MN-major
+        auto issue_kv = [&](uint32_t a_col, uint32_t b_base, uint32_t d_col, bool acc) {
 #pragma unroll
-          for (int kk = 0; kk < kBMq / 16; ++kk) {
-            umma_ss(tmem + col, sw128_desc(a_base + kk * 32, 16, 1024),
-                    sw128_desc(b_base + kk * 2048, C::kQSub, 1024), C::kIdescKV, (acc || kk > 0) ? 1u : 0u);
-          }
+          for (int kk = 0; kk < kBMq / 16; ++kk)
+            umma_ts(tmem + d_col, tmem + a_col + ts_col(kk), sw128_desc(b_base + kk * 2048, C::kSub, 1024),
+                    C::kIdescKV, (acc || kk > 0) ? 1u : 0u);
         };
         bool ok = wait_bar(&bars->kv_full, 0, w, 11) && wait_bar(&bars->q_full[0], 0, w, 12);
         if (ok) {
           tc_fence_after();
-          issue_s(sK, sQ, C::kColS);
+          issue_s(sK, sQ, C::kColR1);
           umma_commit(&bars->s_full);
-          issue_s(sV, sDO, C::kColDP);
+          issue_s(sV, sDO, C::kColR2);
           umma_commit(&bars->dp_full);
         }
-        for (int it = 0; ok && it < nq; ++it) {
-          const int st = it % kStages;
-          const int st1 = (it + 1) % kStages;
-          const bool more = it + 1 < nq;
-          if (!(ok = wait_bar(&bars->pt_ready, it & 1, w, 13))) break;
+        // per tile: dV_i dK_i dQ_i S_{i+1} dP_{i+1}
+        for (int i = 0; ok && i < nq; ++i) {
+          const int st = i % kStages;
+          const uint32_t par = i & 1;
+          if (!(ok = wait_bar(&bars->pt_ready, par, w, 13))) break;
           tc_fence_after();
-          issue_kv(sPt, sDO + st * C::kQBytes, C::kColDV, it > 0);
-          if (more) {
-            if (!(ok = wait_bar(&bars->q_full[st1], ((it + 1) / kStages) & 1, w, 14))) break;
-            tc_fence_after();
-            issue_s(sK, sQ + st1 * C::kQBytes, C::kColS);
-            umma_commit(&bars->s_full);
-          }
-          if (!(ok = wait_bar(&bars->ds_ready, it & 1, w, 15))) break;
+          issue_kv(C::kColR1, sDO + st * C::kTile, C::kColDV, i > 0);
+          umma_commit(&bars->dv_done);
+          if (!(ok = wait_bar(&bars->ds_ready, par, w, 15))) break;
           tc_fence_after();
-          issue_kv(sDSt, sQ + st * C::kQBytes, C::kColDK, it > 0);
-          umma_commit(&bars->q_empty[st]);
-          const int buf = it & 1;
-          if (it >= 2 && !(ok = wait_bar(&bars->dq_free[buf], ((it - 2) >> 1) & 1, w, 16))) break;
-          tc_fence_after();
-          // dQ^T = K^T dS^T: A = K as [128 d (M, contiguous)][128 keys], B = dS^T as [64 q (N, contiguous)][128 keys]
+          issue_kv(C::kColR2, sQ + st * C::kTile, C::kColDK, i > 0);
+          // dQ^T = K^T dS^T over R2: A = K as [128 d (M, contiguous)][128 keys], B = dS^T as
+          // [128 q (N, contiguous)][128 keys] in the dO stage buffer
+          const uint32_t ds = sDO + st * C::kTile;
 #pragma unroll
-          for (int kk = 0; kk < kBN / 16; ++kk) {
-            umma_ss(tmem + C::kColDQ + buf * 64, sw128_desc(sK + kk * 2048, C::kKVSub, 1024),
-                    sw128_desc(sDSt + kk * 2048, C::kKVSub, 1024), C::kIdescQ, kk > 0 ? 1u : 0u);
-          }
-          umma_commit(&bars->dq_full[buf]);
-          if (more) {
-            issue_s(sV, sDO + st1 * C::kQBytes, C::kColDP);
+          for (int kk = 0; kk < kBN / 16; ++kk)
+            umma_ss(tmem + C::kColR2, sw128_desc(sK + kk * 2048, C::kSub, 1024),
+                    sw128_desc(ds + kk * 2048, C::kSub, 1024), C::kIdescQ, kk > 0 ? 1u : 0u);
+          umma_commit(&bars->dq_full);
+          umma_commit(&bars->q_empty[st]);
+          if (i + 1 < nq) {
+            const int st1 = (i + 1) % kStages;
+            if (!(ok = wait_bar(&bars->q_full[st1], ((i + 1) / kStages) & 1, w, 14))) break;
+            tc_fence_after();
+            issue_s(sK, sQ + st1 * C::kTile, C::kColR1);
+            umma_commit(&bars->s_full);
+            // dP_{i+1} overwrites dQ_i^T in R2: the drain must have read it
+            if (!(ok = wait_bar(&bars->dq_free, par, w, 16))) break;
+            tc_fence_after();
+            issue_s(sV, sDO + st1 * C::kTile, C::kColR2);
             umma_commit(&bars->dp_full);
           }
         }
@@ -444,7 +512,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   __syncthreads();
-  if (warp == 9) {
+  if (warp == 13) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
@@ -465,12 +533,13 @@ cudaError_t launch_bwd_pre(const BwdArgs& a, cudaStream_t s) {
 }
 
 cudaError_t launch_bwd_main(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                            const CUtensorMap& tdo, const BwdArgs& a, const DevCtl& c, cudaStream_t s) {
+                            const CUtensorMap& tdo, const CUtensorMap& tdq, const BwdArgs& a, const DevCtl& c,
+                            cudaStream_t s) {
   constexpr int smem = BwdCfg::kSmemBytes;
   cudaError_t e = cudaFuncSetAttribute(bwd_main_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   const dim3 grid((a.N + kBN - 1) / kBN, a.H, a.B);
-  bwd_main_kernel<<<grid, kThreads, smem, s>>>(tq, tk, tv, tdo, a, c);
+  bwd_main_kernel<<<grid, kThreads, smem, s>>>(tq, tk, tv, tdo, tdq, a, c);
   return cudaGetLastError();
 }
 

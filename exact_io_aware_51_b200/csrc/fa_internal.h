@@ -46,13 +46,18 @@ struct BwdArgs {
 // positions x 64 features of one (b, h); 128-byte swizzle.
 CUresult make_tile_map(CUtensorMap* map, const void* base, int B, int N, int H, int d, int rows);
 
+// TMA descriptor for the fp32 [B, N, H, d] dQ accumulator with a box of 64
+// sequence positions x d features of one (b, h), no swizzle (for TMA reduce-add).
+CUresult make_dq_accum_map(CUtensorMap* map, float* base, int B, int N, int H, int d);
+
 // Kernel launchers (each returns the cudaError_t of the launch).
 cudaError_t launch_fwd_bf16(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const FwdArgs& a, const DevCtl& c, cudaStream_t s);
 cudaError_t launch_fwd_f32(const float* Q, const float* K, const float* V, const FwdArgs& a, cudaStream_t s);
 cudaError_t launch_bwd_pre(const BwdArgs& a, cudaStream_t s);
 cudaError_t launch_bwd_main(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                            const CUtensorMap& tdo, const BwdArgs& a, const DevCtl& c, cudaStream_t s);
+                            const CUtensorMap& tdo, const CUtensorMap& tdq, const BwdArgs& a, const DevCtl& c,
+                            cudaStream_t s);
 cudaError_t launch_bwd_dq(const BwdArgs& a, cudaStream_t s);
 
 // Test-only single-tile MMA probe (see fa_debug_umma in the public header).
