@@ -101,14 +101,14 @@ constexpr int kBN = 128;        // keys per CTA (TMEM lanes of S^T, dP^T, dK, dV
 constexpr int kBMq = 128;       // query rows per streamed tile
 constexpr int kThreads = 512;   // WG0, WG1: P / dS for query columns 0-63 / 64-127; WG2: dQ drain; WG3: loader + MMA
 constexpr int kStages = 2;      // Q/dO ring
-// 512 x 128 at launch = 2 x 128 x 168 + 128 x 104 + 128 x 72.  A warpgroup above the
+// 512 x 128 at launch = 2 x 128 x 144 + 128 x 144 + 128 x 80.  A warpgroup above the
 // launch count raises its share (setmaxnreg.inc), one below lowers it
 // (setmaxnreg.dec); the other direction is an illegal instruction.
 constexpr uint32_t kRegLaunch = 128;
-constexpr uint32_t kRegCompute = 168;
-constexpr uint32_t kRegDrain = 104;
-constexpr uint32_t kRegCtrl = 72;
-static_assert(kRegCompute >= kRegLaunch && kRegDrain <= kRegLaunch && kRegCtrl <= kRegLaunch,
+constexpr uint32_t kRegCompute = 144;
+constexpr uint32_t kRegDrain = 144;
+constexpr uint32_t kRegCtrl = 80;
+static_assert(kRegCompute >= kRegLaunch && kRegDrain >= kRegLaunch && kRegCtrl <= kRegLaunch,
               "setmaxnreg direction");
 static_assert(2 * kRegCompute + kRegDrain + kRegCtrl == 4 * kRegLaunch, "register split must match the launch");
 
@@ -360,7 +360,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // the columns); each 64-query half is then written to a shared-memory
     // staging tile [64 q][128 d] and added into the fp32 accumulator in global
     // memory by one TMA reduce-add (whole lines, no per-element atomics).
-    reg_dealloc<kRegDrain>();
+    reg_alloc<kRegDrain>();
     if (bars->abort == 0) {
       const int quarter = warp & 3;
       const int dd = quarter * 32 + lane;  // feature index = TMEM lane of dQ^T
@@ -376,39 +376,31 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++sync_phase;
         return r;
       };
-      // write 64 query rows of dQ^T (this thread's feature) into the staging tile and reduce them
-      auto stage_and_reduce = [&](const uint32_t* v, int q_row0) -> bool {
-        if (issuer) bulk_wait_read_all();  // the previous reduction has read the staging tile
-        if (!drain_sync()) return false;
-#pragma unroll
-        for (int c = 0; c < 64; ++c) stage[c * 128 + dd] = __uint_as_float(v[c]);
-        fence_proxy_async_smem();
-        if (!drain_sync()) return false;
-        if (issuer) {
-          tma_reduce_add_4d(&tmDQ, stage, 0, q_row0, h, b);
-          bulk_commit();
-        }
-        return true;
-      };
       for (int i = 0; ok && i < nq; ++i) {
         if (!(ok = warp_all(wait_bar(&bars->dq_full, i & 1, w, 30)))) break;
         tc_fence_after();
         const int q0 = qtile(i) * kBMq;
-        uint32_t v[64];
-        tmem_ld32(tQ, v);
-        tmem_ld32(tQ + 32, v + 32);
+        uint32_t v[kBMq];
+#pragma unroll
+        for (int c = 0; c < kBMq / 32; ++c) tmem_ld32(tQ + 32 * c, v + 32 * c);
         tmem_wait_ld();
-        reg_fence32(v);
-        reg_fence32(v + 32);
-        if (!(ok = stage_and_reduce(v, q0))) break;
-        tmem_ld32(tQ + 64, v);
-        tmem_ld32(tQ + 96, v + 32);
-        tmem_wait_ld();
-        reg_fence32(v);
-        reg_fence32(v + 32);
+#pragma unroll
+        for (int c = 0; c < kBMq / 32; ++c) reg_fence32(v + 32 * c);
         tc_fence_before();
-        mbar_arrive(&bars->dq_free);
-        ok = stage_and_reduce(v, q0 + 64);
+        mbar_arrive(&bars->dq_free);  // dP_{i+1} may overwrite the columns now
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          if (issuer) bulk_wait_read_all();  // the previous reduction has read the staging tile
+          if (!(ok = drain_sync())) break;
+#pragma unroll
+          for (int c = 0; c < 64; ++c) stage[c * 128 + dd] = __uint_as_float(v[64 * half + c]);
+          fence_proxy_async_smem();
+          if (!(ok = drain_sync())) break;
+          if (issuer) {
+            tma_reduce_add_4d(&tmDQ, stage, 0, q0 + 64 * half, h, b);
+            bulk_commit();
+          }
+        }
       }
       if (issuer) bulk_wait_all();
     }
@@ -471,14 +463,24 @@ __global__ void __launch_bounds__(kThreads, 1)
           issue_s(sV, sDO, C::kColR2);
           umma_commit(&bars->dp_full);
         }
-        // per tile: dV_i dK_i dQ_i S_{i+1} dP_{i+1}
+        // per tile: dV_i S_{i+1} dK_i dQ_i dP_{i+1}.  S_{i+1} goes right behind dV_i
+        // (which reads P^T_i from the same columns; the tensor pipe keeps issue
+        // order), so the softmax warps find it ready when they finish tile i.
         for (int i = 0; ok && i < nq; ++i) {
           const int st = i % kStages;
+          const int st1 = (i + 1) % kStages;
           const uint32_t par = i & 1;
+          const bool more = i + 1 < nq;
           if (!(ok = wait_bar(&bars->pt_ready, par, w, 13))) break;
           tc_fence_after();
           issue_kv(C::kColR1, sDO + st * C::kTile, C::kColDV, i > 0);
           umma_commit(&bars->dv_done);
+          if (more) {
+            if (!(ok = wait_bar(&bars->q_full[st1], ((i + 1) / kStages) & 1, w, 14))) break;
+            tc_fence_after();
+            issue_s(sK, sQ + st1 * C::kTile, C::kColR1);
+            umma_commit(&bars->s_full);
+          }
           if (!(ok = wait_bar(&bars->ds_ready, par, w, 15))) break;
           tc_fence_after();
           issue_kv(C::kColR2, sQ + st * C::kTile, C::kColDK, i > 0);
@@ -491,12 +493,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     sw128_desc(ds + kk * 2048, C::kSub, 1024), C::kIdescQ, kk > 0 ? 1u : 0u);
           umma_commit(&bars->dq_full);
           umma_commit(&bars->q_empty[st]);
-          if (i + 1 < nq) {
-            const int st1 = (i + 1) % kStages;
-            if (!(ok = wait_bar(&bars->q_full[st1], ((i + 1) / kStages) & 1, w, 14))) break;
-            tc_fence_after();
-            issue_s(sK, sQ + st1 * C::kTile, C::kColR1);
-            umma_commit(&bars->s_full);
+          if (more) {
             // dP_{i+1} overwrites dQ_i^T in R2: the drain must have read it
             if (!(ok = wait_bar(&bars->dq_free, par, w, 16))) break;
             tc_fence_after();
