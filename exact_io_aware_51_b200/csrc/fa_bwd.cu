@@ -34,6 +34,9 @@ namespace fa {
 namespace {
 
 constexpr float kLog2e = 1.4426950408889634f;
+// When > 0, one float4 group of query columns in kPolyEvery takes its
+// exponentials on the FMA pipe (exp2_poly2) instead of the MUFU unit.
+constexpr int kPolyEvery = 0;
 
 // ---------------------------------------------------------------------------
 // 1. preprocess
@@ -259,65 +262,80 @@ __global__ void __launch_bounds__(kThreads, 1)
         reg_fence32(sr + 32);
         const float4* sL = reinterpret_cast<const float4*>(smem + C::kOffL + st * 512 + 256 * g);
         const float4* sD = reinterpret_cast<const float4*>(smem + C::kOffDv + st * 512 + 256 * g);
-        float p[64];
-#pragma unroll
-        for (int c4 = 0; c4 < 16; ++c4) {
-          const float4 l4 = sL[c4];
-          const float2 x0 = ffma2(make_float2(__uint_as_float(sr[4 * c4]), __uint_as_float(sr[4 * c4 + 1])),
-                                  make_float2(sl2, sl2), make_float2(-l4.x, -l4.y));
-          const float2 x1 = ffma2(make_float2(__uint_as_float(sr[4 * c4 + 2]), __uint_as_float(sr[4 * c4 + 3])),
-                                  make_float2(sl2, sl2), make_float2(-l4.z, -l4.w));
-          p[4 * c4 + 0] = ex2(x0.x);
-          p[4 * c4 + 1] = ex2(x0.y);
-          p[4 * c4 + 2] = ex2(x1.x);
-          p[4 * c4 + 3] = ex2(x1.y);
-        }
         const bool need_mask = (q0 + 64 > a.N) || (key0 + kBN > a.N) || (a.causal && q0 < key0 + kBN);
-        if (need_mask) {
+        float p[64];
+        // P = 2^(S^T * scale * log2 e - LSE * log2 e), 32 query columns at a time;
+        // each half's P^T (bf16 pairs, 16 columns) goes to TMEM while the next half
+        // is computed
 #pragma unroll
-          for (int c = 0; c < 64; ++c) {
-            const int q = q0 + c;
-            const bool vis = (q < a.N) && (key < a.N) && (!a.causal || q >= key);
-            if (!vis) p[c] = 0.f;
+        for (int hh = 0; hh < 2; ++hh) {
+#pragma unroll
+          for (int c4 = 8 * hh; c4 < 8 * hh + 8; ++c4) {
+            const float4 l4 = sL[c4];
+            const float2 x0 = ffma2(make_float2(__uint_as_float(sr[4 * c4]), __uint_as_float(sr[4 * c4 + 1])),
+                                    make_float2(sl2, sl2), make_float2(-l4.x, -l4.y));
+            const float2 x1 = ffma2(make_float2(__uint_as_float(sr[4 * c4 + 2]), __uint_as_float(sr[4 * c4 + 3])),
+                                    make_float2(sl2, sl2), make_float2(-l4.z, -l4.w));
+            float2 y0, y1;
+            if (kPolyEvery > 0 && (c4 % (kPolyEvery > 0 ? kPolyEvery : 1)) == kPolyEvery - 1) {
+              y0 = exp2_poly2(x0);
+              y1 = exp2_poly2(x1);
+            } else {
+              y0 = make_float2(ex2(x0.x), ex2(x0.y));
+              y1 = make_float2(ex2(x1.x), ex2(x1.y));
+            }
+            p[4 * c4 + 0] = y0.x;
+            p[4 * c4 + 1] = y0.y;
+            p[4 * c4 + 2] = y1.x;
+            p[4 * c4 + 3] = y1.y;
           }
-        }
-        {  // P^T (bf16 pairs) over the first 32 of this WG's R1 columns
-          uint32_t pk[32];
+          if (need_mask) {
 #pragma unroll
-          for (int c = 0; c < 32; ++c) pk[c] = pack_bf16x2(p[2 * c], p[2 * c + 1]);
-          tmem_st32(tR1, pk);
-          tmem_wait_st();
+            for (int c = 32 * hh; c < 32 * hh + 32; ++c) {
+              const int q = q0 + c;
+              const bool vis = (q < a.N) && (key < a.N) && (!a.causal || q >= key);
+              if (!vis) p[c] = 0.f;
+            }
+          }
+          uint32_t pk[16];
+#pragma unroll
+          for (int c = 0; c < 16; ++c) pk[c] = pack_bf16x2(p[32 * hh + 2 * c], p[32 * hh + 2 * c + 1]);
+          tmem_st16(tR1 + 16 * hh, pk);
         }
+        tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&bars->pt_ready);
 
         ok = warp_all(wait_bar(&bars->dp_full, par, w, 22));
         if (!ok) break;
-        tc_fence_after();
-        uint32_t dr[64];
-        tmem_ld32(tR2, dr);
-        tmem_ld32(tR2 + 32, dr + 32);
-        tmem_wait_ld();
-        reg_fence32(dr);
-        reg_fence32(dr + 32);
-        uint32_t pk[32];
-#pragma unroll
-        for (int c4 = 0; c4 < 16; ++c4) {
-          const float4 d4 = sD[c4];
-          pk[2 * c4] = pack_bf16x2(p[4 * c4 + 0] * (__uint_as_float(dr[4 * c4 + 0]) - d4.x),
-                                   p[4 * c4 + 1] * (__uint_as_float(dr[4 * c4 + 1]) - d4.y));
-          pk[2 * c4 + 1] = pack_bf16x2(p[4 * c4 + 2] * (__uint_as_float(dr[4 * c4 + 2]) - d4.z),
-                                       p[4 * c4 + 3] * (__uint_as_float(dr[4 * c4 + 3]) - d4.w));
-        }
-        // dS^T into TMEM (A operand of dK) ...
-        tmem_st32(tR2, pk);
-        // ... and into shared memory over dO_i (B operand of dQ^T) once dV_i has read dO_i
+        // dS^T also goes to shared memory over dO_i, which dV_i must have read
         ok = warp_all(wait_bar(&bars->dv_done, par, w, 24));
         if (!ok) break;
+        tc_fence_after();
         const uint32_t sDSt = smem_u32(smem + C::kOffDO + st * C::kTile + g * C::kSub);
+        // dS = P (dP - D), 32 query columns at a time: to TMEM (A operand of dK)
+        // and to shared memory (B operand of dQ^T)
 #pragma unroll
-        for (int u = 0; u < 8; ++u)
-          st_shared_v4(sDSt + sw128_offset(r, u), pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+        for (int hh = 0; hh < 2; ++hh) {
+          uint32_t dr[32];
+          tmem_ld32(tR2 + 32 * hh, dr);
+          tmem_wait_ld();
+          reg_fence32(dr);
+          uint32_t pk[16];
+#pragma unroll
+          for (int c4 = 0; c4 < 8; ++c4) {
+            const float4 d4 = sD[8 * hh + c4];
+            const int c = 32 * hh + 4 * c4;
+            pk[2 * c4] = pack_bf16x2(p[c + 0] * (__uint_as_float(dr[4 * c4 + 0]) - d4.x),
+                                     p[c + 1] * (__uint_as_float(dr[4 * c4 + 1]) - d4.y));
+            pk[2 * c4 + 1] = pack_bf16x2(p[c + 2] * (__uint_as_float(dr[4 * c4 + 2]) - d4.z),
+                                         p[c + 3] * (__uint_as_float(dr[4 * c4 + 3]) - d4.w));
+          }
+          tmem_st16(tR2 + 16 * hh, pk);
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            st_shared_v4(sDSt + sw128_offset(r, 4 * hh + u), pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+        }
         fence_proxy_async_smem();
         tmem_wait_st();
         tc_fence_before();

@@ -50,27 +50,6 @@ constexpr float kTau = 8.0f;    // lazy-rescale threshold (log2 units)
 // were 6-10% slower than none), so it is off.
 constexpr int kPolyEvery = 0;
 
-// 2^x for a pair on the FMA/ALU pipes: x = n + f with n = round(x) (taken by
-// adding and subtracting 1.5 * 2^23) and f in [-1/2, 1/2]; 2^f from a degree-3
-// polynomial with minimal maximum relative error (7.5e-5) on that interval,
-// fitted by the Remez exchange algorithm in gen_exp2_poly.py; 2^n is added to
-// the exponent bits.  x is clamped below at -125 (2^-125 is zero for P after
-// the bf16 rounding), which also maps -inf (masked scores) to that floor.
-__device__ __forceinline__ float2 exp2_poly2(float2 x) {
-  constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
-  x.x = fmaxf(x.x, -125.f);
-  x.y = fmaxf(x.y, -125.f);
-  const float2 t = fadd2(x, make_float2(kShift, kShift));
-  const float2 n = fadd2(t, make_float2(-kShift, -kShift));
-  const float2 f = fadd2(x, make_float2(-n.x, -n.y));
-  float2 p = ffma2(make_float2(5.517166853e-02f, 5.517166853e-02f), f, make_float2(2.426111251e-01f, 2.426111251e-01f));
-  p = ffma2(p, f, make_float2(6.932609677e-01f, 6.932609677e-01f));
-  p = ffma2(p, f, make_float2(9.999280572e-01f, 9.999280572e-01f));
-  const uint32_t ex = __float_as_uint(t.x) << 23;
-  const uint32_t ey = __float_as_uint(t.y) << 23;
-  return make_float2(__uint_as_float(__float_as_uint(p.x) + ex), __uint_as_float(__float_as_uint(p.y) + ey));
-}
-
 template <int D>
 struct FwdCfg {
   static constexpr int kSub = D / 64;                 // 64-feature sub-tiles per row
