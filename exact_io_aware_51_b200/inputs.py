@@ -6,7 +6,7 @@ it without sharing any of the method.
 
 Recipe (the same for every workload): a CPU ``torch.Generator`` seeded with
 ``seed`` draws float32 standard normals of shape [B, N, H, d] in the order
-Q, K, V, dO.  For the long-sequence workload a further ``randperm(N)`` from the
+Q, K, V, dO (K and V with Hkv heads instead of H for grouped-query problems).  For the long-sequence workload a further ``randperm(N)`` from the
 same generator picks floor(frac * N) sequence positions whose K rows (all
 batches and heads) are multiplied by ``spike`` in float32, which forces large
 jumps of the running row maximum in the online softmax.  The tensors are then
@@ -36,6 +36,11 @@ class Workload:
     spike_frac: float = 0.0       # fraction of K rows scaled by ``spike``
     spike: float = 3.0
     seed: int = 0
+    Hkv: int = 0                  # K/V heads (0: same as H)
+
+    @property
+    def kv_heads(self) -> int:
+        return self.Hkv or self.H
 
     def flops_fwd(self, causal: bool) -> float:
         """4*B*H*N^2*d, halved when causal (the usual attention count)."""
@@ -55,7 +60,11 @@ SWEEP = tuple(
     for (b, h, n, d) in ((16, 16, 512, 64), (8, 16, 1024, 128), (4, 32, 2048, 128),
                          (2, 32, 8192, 128), (1, 16, 32768, 128))
 )
-ALL = (FP32_SMALL, BF16_FWD_N1K, BF16_FWDBWD_N4K, BF16_FWDBWD_N16K) + SWEEP
+# Grouped-query attention with the head grouping of the pages' example (64
+# query heads sharing 8 K/V heads).
+BF16_GQA_H64_KV8 = Workload("bf16 fwd+bwd GQA B1 H64 Hkv8 N4096 d128", 1, 64, 4096, 128, "bf16",
+                            (False, True), backward=True, Hkv=8, seed=5)
+ALL = (FP32_SMALL, BF16_FWD_N1K, BF16_FWDBWD_N4K, BF16_FWDBWD_N16K) + SWEEP + (BF16_GQA_H64_KV8,)
 
 
 def torch_dtype(name: str) -> torch.dtype:
@@ -63,17 +72,18 @@ def torch_dtype(name: str) -> torch.dtype:
 
 
 def make_inputs(B: int, N: int, H: int, d: int, *, seed: int = 0, dtype: str = "bf16",
-                spike_frac: float = 0.0, spike: float = 3.0, with_do: bool = True):
-    """Return CPU tensors (q, k, v, do) of shape [B, N, H, d] in ``dtype``.
+                spike_frac: float = 0.0, spike: float = 3.0, with_do: bool = True, kv_heads: int | None = None):
+    """Return CPU tensors (q, k, v, do) in ``dtype``: q, do [B, N, H, d]; k, v [B, N, kv_heads, d].
 
-    ``do`` is None when ``with_do`` is False (it is still drawn, so Q, K, V
-    are the same either way).
+    ``kv_heads`` defaults to H.  ``do`` is None when ``with_do`` is False (it
+    is still drawn, so Q, K, V are the same either way).
     """
     g = torch.Generator(device="cpu").manual_seed(int(seed))
     shape = (B, N, H, d)
+    kv_shape = (B, N, H if kv_heads is None else kv_heads, d)
     q = torch.randn(shape, generator=g, dtype=torch.float32)
-    k = torch.randn(shape, generator=g, dtype=torch.float32)
-    v = torch.randn(shape, generator=g, dtype=torch.float32)
+    k = torch.randn(kv_shape, generator=g, dtype=torch.float32)
+    v = torch.randn(kv_shape, generator=g, dtype=torch.float32)
     do = torch.randn(shape, generator=g, dtype=torch.float32)
     if spike_frac > 0 and N > 0:
         count = int(math.floor(spike_frac * N))
@@ -90,4 +100,4 @@ def make_inputs(B: int, N: int, H: int, d: int, *, seed: int = 0, dtype: str = "
 def workload_inputs(w: Workload, *, with_do=None):
     return make_inputs(w.B, w.N, w.H, w.d, seed=w.seed, dtype=w.dtype,
                        spike_frac=w.spike_frac, spike=w.spike,
-                       with_do=w.backward if with_do is None else with_do)
+                       with_do=w.backward if with_do is None else with_do, kv_heads=w.kv_heads)

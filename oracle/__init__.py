@@ -12,6 +12,8 @@ from .attention import (  # noqa: F401
     forward,
     forward_head,
     forward_rows_head,
+    hidden_keys,
+    kv_head,
     probs_head,
     scores_head,
 )

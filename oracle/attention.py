@@ -44,7 +44,14 @@ Readings where the pages are silent (all recorded in the design notes):
 * causal masking is top-left aligned (key j visible to query i iff j <= i),
   the only reading with equal query and key lengths;
 * inputs are the exact values the GPU sees (bf16 or fp32 widened to fp64) and
-  ``scale`` is the fp32 value the GPU receives, widened.
+  ``scale`` is the fp32 value the GPU receives, widened;
+* grouped-query attention ("Flash Attention" (karlkratz.de), "Grouped Query
+  Attention") groups consecutive query heads: head h reads K/V head
+  h // (H / Hkv);
+* a sliding window ("Flash Attention" (karlkratz.de), "Sliding Window
+  Attention") is a (left, right) pair: key j is visible to query i when
+  i - left <= j <= i + right; the page's window of 4096 tokens is
+  (4095, 0), the position and the 4095 before it.
 
 ``blocked_forward_head`` restates the pages' online-softmax algorithm (key
 blocks streamed, running row max and sum, rescale when the max grows) and is
@@ -59,6 +66,7 @@ from __future__ import annotations
 import numpy as np
 
 __all__ = [
+    "hidden_keys",
     "scores_head",
     "probs_head",
     "forward_head",
@@ -67,6 +75,7 @@ __all__ = [
     "blocked_forward_head",
     "forward",
     "backward",
+    "kv_head",
 ]
 
 
@@ -75,21 +84,44 @@ def _f64(x) -> np.ndarray:
     return a.astype(np.float64, copy=False)
 
 
-def scores_head(q, k, scale: float, causal: bool) -> np.ndarray:
-    """S = scale * Q K^T for one (batch, head), with the causal mask applied.
+def hidden_keys(rows, nk: int, causal: bool, window=None) -> np.ndarray:
+    """Boolean [len(rows), nk] mask: True where key j is hidden from query row i.
 
-    q: [Nq, d], k: [Nk, d].  Masked entries are -inf.  Query row i sits at
-    sequence position i (top-left alignment), so key j is hidden when j > i.
-    Standard attention as defined in "Flash Attention" (Ultralytics glossary),
-    "Flash Attention и смежные понятия" (the same operation with the full
-    score matrix written out).
+    Query row i sits at sequence position i (top-left alignment).
+    * causal: key j is hidden when j > i.
+    * window = (left, right): key j is visible only when i - left <= j <= i + right;
+      None on a side leaves that side unbounded.  "Flash Attention"
+      (karlkratz.de), section "Sliding Window Attention": each position attends
+      to a fixed neighbourhood; the page's 4096-token window is read as
+      (left, right) = (4095, 0): the position itself and the 4095 before it.
+    """
+    rows = np.asarray(rows, dtype=np.int64)[:, None]
+    cols = np.arange(nk)[None, :]
+    hidden = np.zeros((rows.shape[0], nk), dtype=bool)
+    if causal:
+        hidden |= cols > rows
+    if window is not None:
+        left, right = window
+        if right is not None:
+            hidden |= cols > rows + right
+        if left is not None:
+            hidden |= cols < rows - left
+    return hidden
+
+
+def scores_head(q, k, scale: float, causal: bool, window=None) -> np.ndarray:
+    """S = scale * Q K^T for one (batch, head), with the mask applied.
+
+    q: [Nq, d], k: [Nk, d].  Masked entries are -inf (see ``hidden_keys`` for
+    the causal and sliding-window masks).  Standard attention as defined in
+    "Flash Attention" (Ultralytics glossary), "Flash Attention и смежные
+    понятия" (the same operation with the full score matrix written out).
     """
     q = _f64(q)
     k = _f64(k)
     s = float(scale) * (q @ k.T)
-    if causal:
-        nq, nk = s.shape
-        hidden = np.arange(nk)[None, :] > np.arange(nq)[:, None]
+    if causal or window is not None:
+        hidden = hidden_keys(np.arange(s.shape[0]), s.shape[1], causal, window)
         s = np.where(hidden, -np.inf, s)
     return s
 
@@ -111,7 +143,7 @@ def probs_head(s: np.ndarray):
     return p, lse
 
 
-def forward_head(q, k, v, scale: float, causal: bool):
+def forward_head(q, k, v, scale: float, causal: bool, window=None):
     """O = softmax(scale Q K^T + mask) V and LSE for one (batch, head).
 
     q, k, v: [N, d].  Returns O [N, d] float64 and LSE [N] float64.
@@ -119,12 +151,12 @@ def forward_head(q, k, v, scale: float, causal: bool):
     "Flash Attention" (karlkratz.de), "Speicherbedarf und Laufzeitverhalten"
     (same result, not an approximation).
     """
-    s = scores_head(q, k, scale, causal)
+    s = scores_head(q, k, scale, causal, window)
     p, lse = probs_head(s)
     return p @ _f64(v), lse
 
 
-def forward_rows_head(q, k, v, rows, scale: float, causal: bool):
+def forward_rows_head(q, k, v, rows, scale: float, causal: bool, window=None):
     """Forward restricted to the query rows ``rows`` of one (batch, head).
 
     A row of O and its LSE depend only on that query row and all of K and V,
@@ -135,14 +167,13 @@ def forward_rows_head(q, k, v, rows, scale: float, causal: bool):
     q = _f64(q)
     k = _f64(k)
     s = float(scale) * (q[rows] @ k.T)
-    if causal:
-        hidden = np.arange(k.shape[0])[None, :] > rows[:, None]
-        s = np.where(hidden, -np.inf, s)
+    if causal or window is not None:
+        s = np.where(hidden_keys(rows, k.shape[0], causal, window), -np.inf, s)
     p, lse = probs_head(s)
     return p @ _f64(v), lse
 
 
-def backward_head(q, k, v, do, scale: float, causal: bool):
+def backward_head(q, k, v, do, scale: float, causal: bool, window=None):
     """Gradients (dQ, dK, dV) of O = attention(Q, K, V) given dO, one head.
 
     Recomputes S and P from Q, K and V ("Flash Attention" (karlkratz.de),
@@ -153,7 +184,7 @@ def backward_head(q, k, v, do, scale: float, causal: bool):
     k = _f64(k)
     v = _f64(v)
     do = _f64(do)
-    s = scores_head(q, k, scale, causal)
+    s = scores_head(q, k, scale, causal, window)
     p, _ = probs_head(s)
     o = p @ v
     dv = p.T @ do
@@ -219,35 +250,65 @@ def blocked_forward_head(q, k, v, scale: float, causal: bool, block: int,
     return out.astype(dtype), lse.astype(dtype)
 
 
-def forward(Q, K, V, scale: float, causal: bool, heads=None):
-    """Batched forward over [B, N, H, d] tensors (numpy or CPU torch).
+def kv_head(h: int, n_heads: int, n_kv_heads: int) -> int:
+    """K/V head read by query head ``h`` under grouped-query attention.
+
+    "Flash Attention" (karlkratz.de), section "Grouped Query Attention":
+    several query heads share one K/V group (64 query heads on 8 K/V heads in
+    the page's example).  The page does not fix which heads share; the reading
+    taken is consecutive groups, query head h -> K/V head h // (H / Hkv), so
+    Hkv = H is ordinary multi-head attention and Hkv = 1 multi-query attention.
+    """
+    if n_kv_heads < 1 or n_heads % n_kv_heads:
+        raise ValueError("the K/V head count must divide the query head count")
+    return h // (n_heads // n_kv_heads)
+
+
+def forward(Q, K, V, scale: float, causal: bool, heads=None, window=None):
+    """Batched forward: Q [B, N, H, d]; K, V [B, N, Hkv, d] (numpy or CPU torch).
 
     Returns O [B, N, H, d] and LSE [B, H, N] in float64.  ``heads`` restricts
-    the work to a list of (b, h) pairs; other entries are left as NaN.
+    the work to a list of (b, h) query-head pairs; other entries are left as
+    NaN.  With Hkv < H each query head attends with K/V head ``kv_head(h)``.
     """
     Q, K, V = (_f64(_to_numpy(t)) for t in (Q, K, V))
     b_, n_, h_, d_ = Q.shape
+    hkv = K.shape[2]
     O = np.full((b_, n_, h_, V.shape[3]), np.nan)
     LSE = np.full((b_, h_, n_), np.nan)
     for (b, h) in (heads if heads is not None else _all_heads(b_, h_)):
-        o, lse = forward_head(Q[b, :, h], K[b, :, h], V[b, :, h], scale, causal)
+        g = kv_head(h, h_, hkv)
+        o, lse = forward_head(Q[b, :, h], K[b, :, g], V[b, :, g], scale, causal, window)
         O[b, :, h] = o
         LSE[b, h] = lse
     return O, LSE
 
 
-def backward(Q, K, V, dO, scale: float, causal: bool, heads=None):
-    """Batched backward over [B, N, H, d].  Returns dQ, dK, dV (float64)."""
+def backward(Q, K, V, dO, scale: float, causal: bool, heads=None, window=None):
+    """Batched backward.  Returns dQ [B, N, H, d], dK and dV [B, N, Hkv, d] (float64).
+
+    A K/V head shared by a group of query heads enters each of their
+    attentions, so its gradient is the sum of the per-query-head gradients
+    (chain rule).  With ``heads`` given, dK and dV sum over the listed query
+    heads only (entries no listed head touches stay NaN).
+    """
     Q, K, V, dO = (_f64(_to_numpy(t)) for t in (Q, K, V, dO))
     shape = Q.shape
+    hkv = K.shape[2]
     dQ = np.full(shape, np.nan)
-    dK = np.full(shape, np.nan)
+    dK = np.full(K.shape, np.nan)
     dV = np.full(V.shape, np.nan)
+    touched = set()
     for (b, h) in (heads if heads is not None else _all_heads(shape[0], shape[2])):
-        dq, dk, dv, _ = backward_head(Q[b, :, h], K[b, :, h], V[b, :, h], dO[b, :, h], scale, causal)
+        g = kv_head(h, shape[2], hkv)
+        dq, dk, dv, _ = backward_head(Q[b, :, h], K[b, :, g], V[b, :, g], dO[b, :, h], scale, causal, window)
         dQ[b, :, h] = dq
-        dK[b, :, h] = dk
-        dV[b, :, h] = dv
+        if (b, g) not in touched:
+            touched.add((b, g))
+            dK[b, :, g] = 0.0
+            dV[b, :, g] = 0.0
+        dK[b, :, g] += dk
+        dV[b, :, g] += dv
     return dQ, dK, dV
 
 

@@ -173,6 +173,122 @@ def pin_autograd(bwd=A.backward_head, fwd=A.forward_head):
     return worst
 
 
+def _gqa_case(seed, B=2, N=19, H=6, Hkv=2, d=4):
+    q = _rand((B, N, H, d), seed)
+    k = _rand((B, N, Hkv, d), seed + 1)
+    v = _rand((B, N, Hkv, d), seed + 2)
+    do = _rand((B, N, H, d), seed + 3)
+    return q, k, v, do
+
+
+def pin_gqa_torch(fwd=A.forward, bwd=A.backward):
+    """Grouped-query attention against torch's SDPA with enable_gqa (fp64, CPU, autograd).
+
+    torch repeats each K/V head over H / Hkv consecutive query heads, the
+    grouping read from "Flash Attention" (karlkratz.de), "Grouped Query Attention".
+    """
+    worst = 0.0
+    for causal in (False, True):
+        for H, Hkv in ((6, 2), (6, 1), (4, 4)):
+            q, k, v, do = _gqa_case(60 + H + Hkv, H=H, Hkv=Hkv)
+            tq, tk, tv = (torch.tensor(x.transpose(0, 2, 1, 3), requires_grad=True) for x in (q, k, v))
+            out = torch.nn.functional.scaled_dot_product_attention(
+                tq, tk, tv, is_causal=causal, scale=0.6, enable_gqa=True)
+            out.backward(torch.tensor(do.transpose(0, 2, 1, 3)))
+            o, _ = fwd(q, k, v, 0.6, causal)
+            dq, dk, dv = bwd(q, k, v, do, 0.6, causal)
+            pairs = ((o, out.detach()), (dq, tq.grad), (dk, tk.grad), (dv, tv.grad))
+            for a, b in pairs:
+                worst = max(worst, float(np.max(np.abs(a - b.numpy().transpose(0, 2, 1, 3)))))
+    return worst
+
+
+def pin_gqa_finite_differences(bwd=A.backward, causal=True):
+    """dK, dV of a shared K/V head by central differences of L = sum(O * dO) over all query heads."""
+    q, k, v, do = _gqa_case(70, B=1, N=9, H=6, Hkv=2, d=3)
+    dq, dk, dv = bwd(q, k, v, do, 0.8, causal)
+
+    def loss(kk, vv):
+        o, _ = A.forward(q, kk, vv, 0.8, causal)
+        return float(np.sum(o * do))
+
+    eps = 1e-6
+    worst = 0.0
+    for (n, g, c) in ((0, 0, 0), (4, 1, 2), (8, 0, 1), (3, 1, 0)):
+        for which, grad in (("k", dk), ("v", dv)):
+            kp, km = k.copy(), k.copy()
+            vp, vm = v.copy(), v.copy()
+            if which == "k":
+                kp[0, n, g, c] += eps
+                km[0, n, g, c] -= eps
+            else:
+                vp[0, n, g, c] += eps
+                vm[0, n, g, c] -= eps
+            fd = (loss(kp, vp) - loss(km, vm)) / (2 * eps)
+            worst = max(worst, abs(fd - grad[0, n, g, c]))
+    return worst
+
+
+WINDOWS = ((0, 0), (1, 0), (3, 2), (0, 4), (None, 0), (5, None), (None, None), (2, 40))
+
+
+def pin_window_rowwise(fwd=A.forward_head):
+    """Sliding window: each row is ordinary softmax attention over the slice of
+    keys k[i-left : i+right+1] (the neighbourhood itself, no mask involved)."""
+    n, d = 23, 4
+    q, k, v = _rand((n, d), 90), _rand((n, d), 91), _rand((n, 3), 92)
+    worst = 0.0
+    for window in WINDOWS:
+        o, lse = fwd(q, k, v, 0.7, False, window)
+        left, right = window
+        for i in range(n):
+            lo = 0 if left is None else max(0, i - left)
+            hi = n if right is None else min(n, i + right + 1)
+            s = 0.7 * (k[lo:hi] @ q[i])
+            e = np.exp(s - s.max())
+            worst = max(worst, float(np.max(np.abs(o[i] - e @ v[lo:hi] / e.sum()))),
+                        abs(lse[i] - (s.max() + math.log(e.sum()))))
+    return worst
+
+
+def pin_window_zero_width(fwd=A.forward_head):
+    """Window (0, 0) leaves one key per row: O_i = v_i and LSE_i = scale <q_i, k_i>."""
+    n, d = 11, 5
+    q, k, v = _rand((n, d), 93), _rand((n, d), 94), _rand((n, d), 95)
+    o, lse = fwd(q, k, v, 0.3, False, (0, 0))
+    return float(max(np.max(np.abs(o - v)), np.max(np.abs(lse - 0.3 * np.sum(q * k, axis=1)))))
+
+
+def pin_window_finite_differences(bwd=A.backward_head, window=(2, 1)):
+    """Central differences of L = sum(dO * O) under a sliding window."""
+    n, d = 7, 3
+    q, k, v, do = (_rand((n, d), s) for s in (96, 97, 98, 99))
+    dq, dk, dv, _ = bwd(q, k, v, do, 0.8, False, window)
+    h = 1e-6
+    worst = 0.0
+    for which, grad in ((0, dq), (1, dk), (2, dv)):
+        for idx in np.ndindex(n, d):
+            args = [q.copy(), k.copy(), v.copy()]
+            args[which][idx] += h
+            lp = float(np.sum(do * A.forward_head(*args, 0.8, False, window)[0]))
+            args[which][idx] -= 2 * h
+            lm = float(np.sum(do * A.forward_head(*args, 0.8, False, window)[0]))
+            worst = max(worst, abs((lp - lm) / (2 * h) - grad[idx]))
+    return worst
+
+
+def window_skipped_block_fraction(n, window, block, hidden=A.hidden_keys):
+    """Fraction of the n x n grid of block x block tiles in which every key is hidden."""
+    skipped = 0
+    for r0 in range(0, n, block):
+        h = hidden(np.arange(r0, min(n, r0 + block)), n, False, window)
+        visible_cols = ~np.all(h, axis=0)
+        per_tile = visible_cols.reshape(-1, block).any(axis=1)
+        skipped += int(np.sum(~per_tile))
+    nb = n // block
+    return skipped / (nb * nb)
+
+
 # ---------------------------------------------------------------------------
 # The pins themselves
 # ---------------------------------------------------------------------------
@@ -385,3 +501,126 @@ def test_backward_mutants_are_caught(kind):
     b = _mut_bwd(kind)
     fails = [_caught(lambda g, c=c: pin_finite_differences(bwd=g, causal=c), b) for c in (False, True)]
     assert any(fails), kind
+
+
+def test_gqa_matches_torch_enable_gqa():
+    assert pin_gqa_torch() < 1e-12
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_gqa_shared_head_gradient_finite_differences(causal):
+    assert pin_gqa_finite_differences(causal=causal) < 1e-7
+
+
+def test_gqa_with_equal_head_counts_is_multi_head():
+    q, k, v, do = _gqa_case(80, H=3, Hkv=3)
+    o, lse = A.forward(q, k, v, 0.5, True)
+    for h in range(3):
+        oh, lh = A.forward_head(q[1, :, h], k[1, :, h], v[1, :, h], 0.5, True)
+        assert np.array_equal(o[1, :, h], oh) and np.array_equal(lse[1, h], lh)
+    with pytest.raises(ValueError):
+        A.kv_head(0, 6, 4)
+
+
+def _mut_gqa_fwd(interleaved):
+    def fwd(Q, K, V, scale, causal):
+        b_, n_, h_, _ = Q.shape
+        hkv = K.shape[2]
+        O = np.zeros(Q.shape[:3] + (V.shape[3],))
+        for b in range(b_):
+            for h in range(h_):
+                g = h % hkv if interleaved else A.kv_head(h, h_, hkv)
+                O[b, :, h], _ = A.forward_head(Q[b, :, h], K[b, :, g], V[b, :, g], scale, causal)
+        return O, None
+    return fwd
+
+
+def _mut_gqa_bwd(kind):
+    def bwd(Q, K, V, dO, scale, causal):
+        h_, hkv = Q.shape[2], K.shape[2]
+        dQ, dK, dV = np.zeros(Q.shape), np.zeros(K.shape), np.zeros(V.shape)
+        for b in range(Q.shape[0]):
+            for h in range(h_):
+                g = A.kv_head(h, h_, hkv)
+                dq, dk, dv, _ = A.backward_head(Q[b, :, h], K[b, :, g], V[b, :, g], dO[b, :, h], scale, causal)
+                dQ[b, :, h] = dq
+                if kind == "last_head_wins":
+                    dK[b, :, g], dV[b, :, g] = dk, dv
+                elif kind == "group_mean":
+                    dK[b, :, g] += dk / (h_ // hkv)
+                    dV[b, :, g] += dv / (h_ // hkv)
+        return dQ, dK, dV
+    return bwd
+
+
+def test_gqa_mutants_are_caught():
+    # interleaved grouping (h % Hkv) instead of consecutive groups
+    assert _caught(lambda g: pin_gqa_torch(fwd=g), _mut_gqa_fwd(True))
+    assert not _caught(lambda g: pin_gqa_torch(fwd=g), _mut_gqa_fwd(False))
+    for kind in ("last_head_wins", "group_mean"):
+        b = _mut_gqa_bwd(kind)
+        assert _caught(lambda g: pin_gqa_finite_differences(bwd=g), b, tol=1e-7), kind
+        assert _caught(lambda g: pin_gqa_torch(bwd=g), b), kind
+
+
+def test_window_rows_equal_attention_over_their_neighbourhood():
+    assert pin_window_rowwise() < 1e-12
+
+
+def test_window_zero_width_closed_form():
+    assert pin_window_zero_width() < 1e-12
+
+
+def test_window_special_cases_reduce_to_full_and_causal():
+    q, k, v = _rand((19, 4), 100), _rand((19, 4), 101), _rand((19, 4), 102)
+    full = A.forward_head(q, k, v, 0.5, False)
+    causal = A.forward_head(q, k, v, 0.5, True)
+    for a, b in zip(A.forward_head(q, k, v, 0.5, False, (None, None)), full):
+        assert np.array_equal(a, b)
+    for a, b in zip(A.forward_head(q, k, v, 0.5, False, (None, 0)), causal):
+        assert np.array_equal(a, b)
+    # a window wider than the sequence hides nothing
+    for a, b in zip(A.forward_head(q, k, v, 0.5, True, (100, 100)), causal):
+        assert np.array_equal(a, b)
+
+
+def test_window_backward_finite_differences():
+    for window in ((2, 1), (0, 3), (None, 0), (1, None)):
+        assert pin_window_finite_differences(window=window) < 1e-7, window
+
+
+def test_window_skips_the_pages_share_of_blocks():
+    """The page: a 4096-token window over 32768 tokens leaves up to 87 % of the
+    blocks uncomputed.  With the (4095, 0) reading and 128 x 128 blocks the
+    mask hides 87.9 % of the full block grid."""
+    g = json.loads((GOLDEN / "sliding_window_blocks.json").read_text())
+    w = g["window_tokens"]
+    frac = window_skipped_block_fraction(g["N"], (w - 1, 0), g["block"])
+    assert g["skipped_fraction_stated"] <= frac < g["skipped_fraction_stated"] + 0.01
+
+
+def _mut_window(kind):
+    def hidden(rows, nk, causal, window=None):
+        if window is not None and kind == "left_off_by_one":
+            left, right = window
+            window = (None if left is None else left + 1, right)
+        if window is not None and kind == "swapped_sides":
+            window = (window[1], window[0])
+        return A.hidden_keys(rows, nk, causal, window)
+
+    def fwd(q, k, v, scale, causal, window=None):
+        s = scale * (np.asarray(q) @ np.asarray(k).T)
+        s = np.where(hidden(np.arange(s.shape[0]), s.shape[1], causal, window), -np.inf, s)
+        p, lse = A.probs_head(s)
+        return p @ v, lse
+    return fwd, hidden
+
+
+@pytest.mark.parametrize("kind", ["left_off_by_one", "swapped_sides"])
+def test_window_mutants_are_caught(kind):
+    fwd, hidden = _mut_window(kind)
+    assert _caught(pin_window_rowwise, fwd)
+    if kind == "left_off_by_one":
+        frac = window_skipped_block_fraction(32768, (4095, 0), 128, hidden=hidden)
+        assert not (0.87 <= frac < 0.88) or _caught(pin_window_zero_width, fwd)
+
