@@ -33,7 +33,8 @@ _LIB = None
 # Every symbol include/fa.h declares.
 EXPORTED = ("fa_fwd", "fa_bwd_workspace_size", "fa_bwd", "fa_status_string", "fa_last_cuda_error",
             "fa_last_device_status", "fa_set_wait_limit_ms", "fa_debug_inject", "fa_debug_umma",
-            "fa_version", "fa_set_kernel_events", "fa_bwd_static_scratch")
+            "fa_version", "fa_set_kernel_events", "fa_bwd_static_scratch", "fa_fwd_gqa", "fa_bwd_gqa",
+            "fa_fwd_window", "fa_bwd_window")
 
 
 class FAError(RuntimeError):
@@ -67,6 +68,14 @@ def lib() -> ctypes.CDLL:
     L.fa_bwd_workspace_size.restype = sz
     L.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, i, vp, sz, vp]
     L.fa_bwd.restype = i
+    L.fa_fwd_gqa.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp]
+    L.fa_fwd_gqa.restype = i
+    L.fa_bwd_gqa.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp, sz, vp]
+    L.fa_bwd_gqa.restype = i
+    L.fa_fwd_window.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, i, vp]
+    L.fa_fwd_window.restype = i
+    L.fa_bwd_window.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, i, vp, sz, vp]
+    L.fa_bwd_window.restype = i
     L.fa_status_string.argtypes = [i]
     L.fa_status_string.restype = ctypes.c_char_p
     L.fa_last_cuda_error.argtypes = []
@@ -106,33 +115,64 @@ def _stream_handle(stream, device) -> int:
     return s.cuda_stream
 
 
-def _check_inputs(*ts: torch.Tensor):
-    t0 = ts[0]
-    if t0.dim() != 4:
+def _check_inputs(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *qlike: torch.Tensor) -> int:
+    """Validate [B, N, H, d] q (and o, do) against [B, N, Hkv, d] k, v; returns Hkv."""
+    if q.dim() != 4 or k.dim() != 4:
         raise ValueError("expected [B, N, H, d] tensors")
-    if not t0.is_cuda:
-        raise ValueError("tensors must live on a CUDA device (there is no CPU path)")
-    for t in ts:
-        if t.shape != t0.shape or t.dtype != t0.dtype or t.device != t0.device:
-            raise ValueError("q, k, v (and o, do) must share shape, dtype and device")
+    B, N, H, d = q.shape
+    Hkv = k.shape[2]
+    grouped = (Hkv == 0 and H == 0) or (Hkv >= 1 and H % Hkv == 0)  # no heads at all is an empty problem
+    if k.shape != (B, N, Hkv, d) or not grouped:
+        raise ValueError("k, v must be [B, N, Hkv, d] with Hkv dividing the query heads H")
+    for t in (q, k, v, *qlike):
+        want = k.shape if t is k or t is v else q.shape
+        if t.shape != want or t.dtype != q.dtype or t.device != q.device:
+            raise ValueError("q, o, do must share one shape; k, v another; all one dtype and device")
         if not t.is_contiguous():
-            raise ValueError("tensors must be contiguous [B, N, H, d]")
+            raise ValueError("tensors must be contiguous [B, N, heads, d]")
+    if not q.is_cuda:
+        raise ValueError("tensors must live on a CUDA device (there is no CPU path)")
+    return Hkv
 
 
 def _scale(scale, d):
     return float(1.0 / math.sqrt(d)) if scale is None else float(scale)
 
 
-def fwd(q, k, v, causal: bool = False, scale: float | None = None, out=None, lse=None, stream=None):
-    """Forward pass: returns (o [B, N, H, d], lse [B, H, N] fp32)."""
-    _check_inputs(q, k, v)
+def _window_bounds(causal, window):
+    """(left, right) bounds for fa_*_window: None -> -1 (open); causal closes the right side at 0."""
+    left, right = window
+    for x in (left, right):
+        if x is not None and (int(x) != x or x < 0):
+            raise ValueError("window bounds must be None or integers >= 0")
+    if causal:
+        right = 0 if right is None else min(int(right), 0)
+    return (-1 if left is None else int(left)), (-1 if right is None else int(right))
+
+
+def fwd(q, k, v, causal: bool = False, scale: float | None = None, out=None, lse=None, stream=None,
+        window=None):
+    """Forward pass: returns (o [B, N, H, d], lse [B, H, N] fp32).
+
+    k and v may have fewer heads than q (grouped-query attention, fa_fwd_gqa).
+    ``window`` = (left, right) restricts query i to keys i - left .. i + right
+    (None on a side: open), fa_fwd_window.
+    """
+    Hkv = _check_inputs(q, k, v)
     B, N, H, d = q.shape
     o = torch.empty_like(q) if out is None else out
     l = torch.empty((B, H, N), dtype=torch.float32, device=q.device) if lse is None else lse
-    rc = lib().fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), l.data_ptr(), B, H, N, d,
-                      _scale(scale, d), int(bool(causal)), _dtype_code(q), _stream_handle(stream, q.device))
+    tail = (_scale(scale, d), int(bool(causal)), _dtype_code(q), _stream_handle(stream, q.device))
+    ptrs = (q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), l.data_ptr())
+    if window is not None:
+        wl, wr = _window_bounds(causal, window)
+        rc, name = lib().fa_fwd_window(*ptrs, B, H, Hkv, N, d, tail[0], wl, wr, *tail[2:]), "fa_fwd_window"
+    elif Hkv == H:
+        rc, name = lib().fa_fwd(*ptrs, B, H, N, d, *tail), "fa_fwd"
+    else:
+        rc, name = lib().fa_fwd_gqa(*ptrs, B, H, Hkv, N, d, *tail), "fa_fwd_gqa"
     if rc != 0:
-        raise FAError(rc, "fa_fwd")
+        raise FAError(rc, name)
     return o, l
 
 
@@ -141,9 +181,14 @@ def bwd_workspace_size(B: int, H: int, N: int, d: int, dtype: int = FA_BF16) -> 
 
 
 def bwd(q, k, v, o, do, lse, causal: bool = False, scale: float | None = None, workspace=None,
-        dq=None, dk=None, dv=None, stream=None):
-    """Backward pass by recomputation: returns (dq, dk, dv), each [B, N, H, d]."""
-    _check_inputs(q, k, v, o, do)
+        dq=None, dk=None, dv=None, stream=None, window=None):
+    """Backward pass by recomputation: returns (dq, dk, dv), shaped like (q, k, v).
+
+    With fewer K/V heads than query heads (fa_bwd_gqa), dk and dv are summed
+    over each K/V head's query-head group.  ``window`` as in ``fwd`` (the same
+    one the forward used), fa_bwd_window.
+    """
+    Hkv = _check_inputs(q, k, v, o, do)
     B, N, H, d = q.shape
     if lse.shape != (B, H, N) or lse.dtype != torch.float32 or not lse.is_contiguous():
         raise ValueError("lse must be a contiguous fp32 [B, H, N] tensor")
@@ -153,12 +198,19 @@ def bwd(q, k, v, o, do, lse, causal: bool = False, scale: float | None = None, w
     need = bwd_workspace_size(B, H, N, d, _dtype_code(q))
     if workspace is None:
         workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
-    rc = lib().fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(), lse.data_ptr(),
-                      dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, N, d, _scale(scale, d),
-                      int(bool(causal)), _dtype_code(q), workspace.data_ptr(), workspace.numel(),
-                      _stream_handle(stream, q.device))
+    ptrs = (q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(), lse.data_ptr(),
+            dq.data_ptr(), dk.data_ptr(), dv.data_ptr())
+    tail = (_scale(scale, d), int(bool(causal)), _dtype_code(q), workspace.data_ptr(), workspace.numel(),
+            _stream_handle(stream, q.device))
+    if window is not None:
+        wl, wr = _window_bounds(causal, window)
+        rc, name = lib().fa_bwd_window(*ptrs, B, H, Hkv, N, d, tail[0], wl, wr, *tail[2:]), "fa_bwd_window"
+    elif Hkv == H:
+        rc, name = lib().fa_bwd(*ptrs, B, H, N, d, *tail), "fa_bwd"
+    else:
+        rc, name = lib().fa_bwd_gqa(*ptrs, B, H, Hkv, N, d, *tail), "fa_bwd_gqa"
     if rc != 0:
-        raise FAError(rc, "fa_bwd")
+        raise FAError(rc, name)
     return dq, dk, dv
 
 
@@ -198,19 +250,20 @@ def debug_umma(a: torch.Tensor, b: torch.Tensor, a_mn_major: int, b_mn_major: in
 
 class _Attention(torch.autograd.Function):
     @staticmethod
-    def forward(ctx, q, k, v, causal, scale):
-        o, lse = fwd(q, k, v, causal=causal, scale=scale)
+    def forward(ctx, q, k, v, causal, scale, window):
+        o, lse = fwd(q, k, v, causal=causal, scale=scale, window=window)
         ctx.save_for_backward(q, k, v, o, lse)
-        ctx.causal, ctx.scale = causal, scale
+        ctx.causal, ctx.scale, ctx.window = causal, scale, window
         return o
 
     @staticmethod
     def backward(ctx, do):
         q, k, v, o, lse = ctx.saved_tensors
-        dq, dk, dv = bwd(q, k, v, o, do.contiguous(), lse, causal=ctx.causal, scale=ctx.scale)
-        return dq, dk, dv, None, None
+        dq, dk, dv = bwd(q, k, v, o, do.contiguous(), lse, causal=ctx.causal, scale=ctx.scale, window=ctx.window)
+        return dq, dk, dv, None, None, None
 
 
-def attention(q, k, v, causal: bool = False, scale: float | None = None):
-    """Differentiable attention over [B, N, H, d] tensors (forward + recomputing backward)."""
-    return _Attention.apply(q, k, v, causal, scale)
+def attention(q, k, v, causal: bool = False, scale: float | None = None, window=None):
+    """Differentiable attention: q [B, N, H, d], k and v [B, N, Hkv, d] (Hkv divides H);
+    optional sliding ``window`` = (left, right)."""
+    return _Attention.apply(q, k, v, causal, scale, window)

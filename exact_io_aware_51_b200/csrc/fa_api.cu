@@ -137,6 +137,32 @@ int check_shape(int B, int H, int N, int d, int dtype) {
   return FA_OK;
 }
 
+// K/V heads: each of the Hkv heads serves H / Hkv query heads.
+int check_kv_heads(int H, int Hkv) {
+  if (Hkv < 0 || Hkv > H) return FA_ERR_INVALID_ARG;
+  if (H > 0 && (Hkv == 0 || H % Hkv != 0)) return FA_ERR_INVALID_ARG;
+  return FA_OK;
+}
+
+// Window bounds: -1 leaves a side unbounded, otherwise 0 <= bound.
+int check_window(int left, int right) {
+  if (left < -1 || right < -1) return FA_ERR_INVALID_ARG;
+  return FA_OK;
+}
+
+// Kernel form of a window: a side with no bound gets kUnbounded, which is
+// above any sequence length the library accepts, so q - wl and q + wr never
+// clip a visible key and never overflow an int.
+constexpr int kUnbounded = 1 << 30;
+static_assert(kMaxN < kUnbounded / 2, "window sentinel must exceed every sequence length");
+
+void set_window(int left, int right, int* wl, int* wr, int* causal) {
+  // a bound at or above the longest sequence hides nothing: same as no bound
+  *wl = (left < 0 || left >= kMaxN) ? kUnbounded : left;
+  *wr = (right < 0 || right >= kMaxN) ? kUnbounded : right;
+  *causal = (*wl == kUnbounded && *wr == 0) ? 1 : 0;
+}
+
 int check_scale(float scale) {
   if (!std::isfinite(scale) || !(scale > 0.f)) return FA_ERR_INVALID_ARG;
   return FA_OK;
@@ -236,10 +262,12 @@ int fa_last_device_status(void* stream, int* detail) {
   return v ? FA_ERR_DEVICE_TIMEOUT : FA_OK;
 }
 
-int fa_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, int B, int H, int N, int d, float scale,
-           int causal, int dtype, void* stream) {
+int fa_fwd_window(const void* Q, const void* K, const void* V, void* O, float* LSE, int B, int H, int Hkv, int N,
+                  int d, float scale, int window_left, int window_right, int dtype, void* stream) {
   int rc = check_shape(B, H, N, d, dtype);
   if (rc) return rc;
+  if ((rc = check_kv_heads(H, Hkv))) return rc;
+  if ((rc = check_window(window_left, window_right))) return rc;
   if ((rc = check_scale(scale))) return rc;
   if (static_cast<long long>(B) * H * N == 0) return FA_OK;
   if (!Q || !K || !V || !O || !LSE) return FA_ERR_INVALID_ARG;
@@ -251,10 +279,11 @@ int fa_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, int
   FwdArgs a;
   a.B = B;
   a.H = H;
+  a.Hkv = Hkv;
   a.N = N;
   a.d = d;
   a.scale_log2 = scale * 1.4426950408889634f;
-  a.causal = causal ? 1 : 0;
+  set_window(window_left, window_right, &a.wl, &a.wr, &a.causal);
   a.O = O;
   a.LSE = LSE;
   cudaError_t e;
@@ -264,8 +293,8 @@ int fa_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, int
     CUtensorMap tq, tk, tv;
     CUresult r;
     if ((r = make_tile_map(&tq, Q, B, N, H, d, 128)) != CUDA_SUCCESS ||
-        (r = make_tile_map(&tk, K, B, N, H, d, 128)) != CUDA_SUCCESS ||
-        (r = make_tile_map(&tv, V, B, N, H, d, 128)) != CUDA_SUCCESS)
+        (r = make_tile_map(&tk, K, B, N, Hkv, d, 128)) != CUDA_SUCCESS ||
+        (r = make_tile_map(&tv, V, B, N, Hkv, d, 128)) != CUDA_SUCCESS)
       return fail_encode(r);
     if (t_ev_start) cudaEventRecord(t_ev_start, s);
     e = launch_fwd_bf16(tq, tk, tv, a, make_ctl(*st), s);
@@ -273,6 +302,16 @@ int fa_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, int
   }
   if (e != cudaSuccess) return fail_cuda(e);
   return FA_OK;
+}
+
+int fa_fwd_gqa(const void* Q, const void* K, const void* V, void* O, float* LSE, int B, int H, int Hkv, int N, int d,
+               float scale, int causal, int dtype, void* stream) {
+  return fa_fwd_window(Q, K, V, O, LSE, B, H, Hkv, N, d, scale, -1, causal ? 0 : -1, dtype, stream);
+}
+
+int fa_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, int B, int H, int N, int d, float scale,
+           int causal, int dtype, void* stream) {
+  return fa_fwd_window(Q, K, V, O, LSE, B, H, H, N, d, scale, -1, causal ? 0 : -1, dtype, stream);
 }
 
 size_t fa_bwd_workspace_size(int B, int H, int N, int d, int dtype) {
@@ -284,11 +323,13 @@ size_t fa_bwd_workspace_size(int B, int H, int N, int d, int dtype) {
   return dq + 2 * rows;
 }
 
-int fa_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO, const float* LSE, void* dQ,
-           void* dK, void* dV, int B, int H, int N, int d, float scale, int causal, int dtype, void* workspace,
-           size_t workspace_bytes, void* stream) {
+int fa_bwd_window(const void* Q, const void* K, const void* V, const void* O, const void* dO, const float* LSE,
+                  void* dQ, void* dK, void* dV, int B, int H, int Hkv, int N, int d, float scale, int window_left,
+                  int window_right, int dtype, void* workspace, size_t workspace_bytes, void* stream) {
   int rc = check_shape(B, H, N, d, dtype);
   if (rc) return rc;
+  if ((rc = check_kv_heads(H, Hkv))) return rc;
+  if ((rc = check_window(window_left, window_right))) return rc;
   if ((rc = check_scale(scale))) return rc;
   if (dtype != FA_BF16 || d != 128) return FA_ERR_UNSUPPORTED;
   if (static_cast<long long>(B) * H * N == 0) return FA_OK;
@@ -306,12 +347,13 @@ int fa_bwd(const void* Q, const void* K, const void* V, const void* O, const voi
   BwdArgs a;
   a.B = B;
   a.H = H;
+  a.Hkv = Hkv;
   a.N = N;
   a.d = d;
   a.Npad = npad;
   a.scale = scale;
   a.scale_log2 = scale * 1.4426950408889634f;
-  a.causal = causal ? 1 : 0;
+  set_window(window_left, window_right, &a.wl, &a.wr, &a.causal);
   a.O = O;
   a.dO = dO;
   a.LSE = LSE;
@@ -329,8 +371,8 @@ int fa_bwd(const void* Q, const void* K, const void* V, const void* O, const voi
   CUresult r;
   if ((r = make_tile_map(&tq, Q, B, N, H, d, 128)) != CUDA_SUCCESS ||
       (r = make_tile_map(&tdo, dO, B, N, H, d, 128)) != CUDA_SUCCESS ||
-      (r = make_tile_map(&tk, K, B, N, H, d, 128)) != CUDA_SUCCESS ||
-      (r = make_tile_map(&tv, V, B, N, H, d, 128)) != CUDA_SUCCESS ||
+      (r = make_tile_map(&tk, K, B, N, Hkv, d, 128)) != CUDA_SUCCESS ||
+      (r = make_tile_map(&tv, V, B, N, Hkv, d, 128)) != CUDA_SUCCESS ||
       (r = make_dq_accum_map(&tdq, a.dQacc, B, N, H, d)) != CUDA_SUCCESS)
     return fail_encode(r);
   cudaError_t e = launch_bwd_pre(a, s);
@@ -342,6 +384,20 @@ int fa_bwd(const void* Q, const void* K, const void* V, const void* O, const voi
   e = launch_bwd_dq(a, s);
   if (e != cudaSuccess) return fail_cuda(e);
   return FA_OK;
+}
+
+int fa_bwd_gqa(const void* Q, const void* K, const void* V, const void* O, const void* dO, const float* LSE,
+               void* dQ, void* dK, void* dV, int B, int H, int Hkv, int N, int d, float scale, int causal, int dtype,
+               void* workspace, size_t workspace_bytes, void* stream) {
+  return fa_bwd_window(Q, K, V, O, dO, LSE, dQ, dK, dV, B, H, Hkv, N, d, scale, -1, causal ? 0 : -1, dtype,
+                       workspace, workspace_bytes, stream);
+}
+
+int fa_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO, const float* LSE, void* dQ,
+           void* dK, void* dV, int B, int H, int N, int d, float scale, int causal, int dtype, void* workspace,
+           size_t workspace_bytes, void* stream) {
+  return fa_bwd_window(Q, K, V, O, dO, LSE, dQ, dK, dV, B, H, H, N, d, scale, -1, causal ? 0 : -1, dtype,
+                       workspace, workspace_bytes, stream);
 }
 
 int fa_debug_umma(const void* A, const void* B, float* D, int N, int K, int a_mn_major, int b_mn_major, int a_tmem,

@@ -197,14 +197,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int lane = lane_id();
 
   const int jt = blockIdx.x;  // key tile
-  const int h = blockIdx.y;
+  const int hk = blockIdx.y;  // K/V head
   const int b = blockIdx.z;
   const int key0 = jt * kBN;
   const int nq_total = (a.N + kBMq - 1) / kBMq;
-  const int i0 = a.causal ? jt : 0;  // first query tile that sees these keys
-  const int nq = max(0, nq_total - i0);
-  auto qtile = [&](int i) { return i0 + i; };
-  const size_t bh = static_cast<size_t>(b) * a.H + h;
+  // query tiles holding every query that sees one of these keys:
+  // q in [key - wr, key + wl] for each key of the tile
+  const int kmax = min(key0 + kBN - 1, a.N - 1);
+  const int i0 = max(0, key0 - a.wr) / kBMq;
+  const int i_end = min(a.N - 1, kmax + a.wl) / kBMq + 1;
+  // Grouped-query attention: the G query heads of this K/V head all add into
+  // this CTA's dK and dV, so the CTA walks (query head, query tile) pairs.
+  const int G = a.H / a.Hkv;
+  const int nq_head = max(0, min(nq_total, i_end) - i0);  // query tiles per query head
+  const int nq = G * nq_head;                 // iterations of this CTA
+  auto qtile = [&](int i) { return i0 + i % nq_head; };
+  auto qhead = [&](int i) { return hk * G + i / nq_head; };
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->kv_full, 1);
@@ -262,7 +270,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         reg_fence32(sr + 32);
         const float4* sL = reinterpret_cast<const float4*>(smem + C::kOffL + st * 512 + 256 * g);
         const float4* sD = reinterpret_cast<const float4*>(smem + C::kOffDv + st * 512 + 256 * g);
-        const bool need_mask = (q0 + 64 > a.N) || (key0 + kBN > a.N) || (a.causal && q0 < key0 + kBN);
+        // every (query, key) pair of this WG's block visible: no mask
+        const bool need_mask =
+            (q0 + 64 > a.N) || (key0 + kBN > a.N) || (key0 + kBN - 1 > q0 + a.wr) || (key0 < q0 + 63 - a.wl);
         float p[64];
         // P = 2^(S^T * scale * log2 e - LSE * log2 e), 32 query columns at a time;
         // each half's P^T (bf16 pairs, 16 columns) goes to TMEM while the next half
@@ -293,7 +303,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int c = 32 * hh; c < 32 * hh + 32; ++c) {
               const int q = q0 + c;
-              const bool vis = (q < a.N) && (key < a.N) && (!a.causal || q >= key);
+              const bool vis = (q < a.N) && (key < a.N) && (key <= q + a.wr) && (key >= q - a.wl);
               if (!vis) p[c] = 0.f;
             }
           }
@@ -345,7 +355,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ok && nq > 0) ok = warp_all(wait_bar(&bars->acc_done, 0, w, 23));
       if (ok) {
         tc_fence_after();
-        const size_t base = ((static_cast<size_t>(b) * a.N + key) * a.H + h) * D;
+        const size_t base = ((static_cast<size_t>(b) * a.N + key) * a.Hkv + hk) * D;
         const uint32_t col = g == 0 ? C::kColDV : C::kColDK;
         const float mul = g == 0 ? 1.f : a.scale;
         __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(g == 0 ? a.dV : a.dK) + base;
@@ -415,7 +425,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           fence_proxy_async_smem();
           if (!(ok = drain_sync())) break;
           if (issuer) {
-            tma_reduce_add_4d(&tmDQ, stage, 0, q0 + 64 * half, h, b);
+            tma_reduce_add_4d(&tmDQ, stage, 0, q0 + 64 * half, qhead(i), b);
             bulk_commit();
           }
         }
@@ -433,18 +443,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_prefetch_desc(&tmDO);
         mbar_arrive_expect_tx(&bars->kv_full, 2 * C::kTile);
         for (int c = 0; c < D / 64; ++c) {
-          tma_load_4d(smem + C::kOffK + c * C::kSub, &tmK, &bars->kv_full, c * 64, key0, h, b);
-          tma_load_4d(smem + C::kOffV + c * C::kSub, &tmV, &bars->kv_full, c * 64, key0, h, b);
+          tma_load_4d(smem + C::kOffK + c * C::kSub, &tmK, &bars->kv_full, c * 64, key0, hk, b);
+          tma_load_4d(smem + C::kOffV + c * C::kSub, &tmV, &bars->kv_full, c * 64, key0, hk, b);
         }
         for (int i = 0; i < nq; ++i) {
           const int st = i % kStages;
           const int n = i / kStages;
           if (i >= kStages && !wait_bar(&bars->q_empty[st], (n - 1) & 1, w, 10)) break;
           const int q0 = qtile(i) * kBMq;
+          const int hq = qhead(i);
+          const size_t bh = static_cast<size_t>(b) * a.H + hq;
           mbar_arrive_expect_tx(&bars->q_full[st], 2 * C::kTile + 1024);
           for (int c = 0; c < D / 64; ++c) {
-            tma_load_4d(smem + C::kOffQ + st * C::kTile + c * C::kSub, &tmQ, &bars->q_full[st], c * 64, q0, h, b);
-            tma_load_4d(smem + C::kOffDO + st * C::kTile + c * C::kSub, &tmDO, &bars->q_full[st], c * 64, q0, h, b);
+            tma_load_4d(smem + C::kOffQ + st * C::kTile + c * C::kSub, &tmQ, &bars->q_full[st], c * 64, q0, hq, b);
+            tma_load_4d(smem + C::kOffDO + st * C::kTile + c * C::kSub, &tmDO, &bars->q_full[st], c * 64, q0, hq,
+                        b);
           }
           bulk_load(smem + C::kOffL + st * 512, a.LSE2 + bh * a.Npad + q0, 512, &bars->q_full[st]);
           bulk_load(smem + C::kOffDv + st * 512, a.Dvec + bh * a.Npad + q0, 512, &bars->q_full[st]);
@@ -553,7 +566,7 @@ cudaError_t launch_bwd_main(const CUtensorMap& tq, const CUtensorMap& tk, const 
   constexpr int smem = BwdCfg::kSmemBytes;
   cudaError_t e = cudaFuncSetAttribute(bwd_main_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  const dim3 grid((a.N + kBN - 1) / kBN, a.H, a.B);
+  const dim3 grid((a.N + kBN - 1) / kBN, a.Hkv, a.B);
   bwd_main_kernel<<<grid, kThreads, smem, s>>>(tq, tk, tv, tdo, tdq, a, c);
   return cudaGetLastError();
 }

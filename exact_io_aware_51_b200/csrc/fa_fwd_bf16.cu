@@ -22,8 +22,11 @@
 //   * lazy rescale: the reference maximum m only moves when a row's maximum
 //     grows by more than 2^8; numerator and denominator share m, so the result
 //     is exact and the O rescale (a TMEM read-modify-write) is rare;
-//   * causal: key tiles beyond the query tile's diagonal are never visited and
-//     only the diagonal tile is masked; CTAs with longer rows start first;
+//   * causal and sliding-window masks: key tiles that no row of the query
+//     tile can see are never loaded or multiplied ("Flash Attention"
+//     (karlkratz.de), "Sliding Window Attention": blocks outside the window
+//     are skipped); only the tiles that straddle the window's edge are masked;
+//     under the causal mask CTAs with longer rows start first;
 //   * epilogue: O / l -> bf16 with 16-byte stores, LSE = (m + log2 l) ln 2.
 // The two query tiles ping-pong: while the softmax of one tile runs, the
 // tensor pipe computes the other tile's products.
@@ -104,14 +107,24 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int cb = a.causal ? (nqb - 1 - static_cast<int>(blockIdx.x)) : static_cast<int>(blockIdx.x);
   const int h = blockIdx.y;
   const int b = blockIdx.z;
-  const int nk_total = (a.N + kBN - 1) / kBN;
-  int q0[2], nkt[2];
+  const int hk = h / (a.H / a.Hkv);  // K/V head of this query head (grouped-query attention)
+  // Key tiles [klo[t], klo[t] + nkt[t]) hold every key some row of query tile
+  // t may see; the CTA streams their union, key tiles kbase .. kbase + nk - 1
+  // (the two ranges overlap or touch, since each row sees its own key).
+  int q0[2], klo[2], nkt[2];
 #pragma unroll
   for (int t = 0; t < 2; ++t) {
     q0[t] = cb * 2 * kBM + t * kBM;
-    nkt[t] = (q0[t] < a.N) ? (a.causal ? min(nk_total, q0[t] / kBN + 1) : nk_total) : 0;
+    klo[t] = 0;
+    nkt[t] = 0;
+    if (q0[t] < a.N) {
+      const int qmax = min(q0[t] + kBM - 1, a.N - 1);
+      klo[t] = max(0, q0[t] - a.wl) / kBN;
+      nkt[t] = min(a.N - 1, qmax + a.wr) / kBN + 1 - klo[t];
+    }
   }
-  const int nk = max(nkt[0], nkt[1]);
+  const int kbase = klo[0];
+  const int nk = (nkt[1] > 0) ? max(klo[0] + nkt[0], klo[1] + nkt[1]) - kbase : nkt[0];
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
@@ -164,13 +177,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int c = 0; c < kBN / 32; ++c) reg_fence32(sr + c * 32);
 
-        const int k0 = j * kBN;
-        const bool need_mask = (a.causal && k0 + kBN - 1 > q0[t]) || (k0 + kBN > a.N);
+        const int k0 = (klo[t] + j) * kBN;
+        // whole tile visible to every row of the query tile: no mask
+        const bool need_mask = (k0 + kBN > a.N) || (k0 + kBN - 1 > q0[t] + a.wr) || (k0 < q0[t] + kBM - 1 - a.wl);
         if (need_mask) {
-          const int lim = a.causal ? min(a.N - 1, qrow) : (a.N - 1);  // last visible key
+          const int hi = min(a.N - 1, qrow + a.wr);  // visible keys: [lo, hi]
+          const int lo = qrow - a.wl;
 #pragma unroll
           for (int c = 0; c < kBN; ++c)
-            if (k0 + c > lim) sr[c] = __float_as_uint(-INFINITY);
+            if (k0 + c > hi || k0 + c < lo) sr[c] = __float_as_uint(-INFINITY);
         }
         float mx0 = __uint_as_float(sr[0]), mx1 = __uint_as_float(sr[1]);
         float mx2 = __uint_as_float(sr[2]), mx3 = __uint_as_float(sr[3]);
@@ -291,12 +306,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive_expect_tx(&bars->k_full[s], C::kTileBytes + extra);
           for (int c = 0; c < C::kSub; ++c)
             tma_load_4d(smem + C::kOffK + s * C::kTileBytes + c * C::kSubBytes, &tmK, &bars->k_full[s], c * 64,
-                        j * kBN, h, b);
+                        (kbase + j) * kBN, hk, b);
           if (j >= C::kStages && !wait_bar(&bars->v_empty[s], (n - 1) & 1, w, 2)) break;
           mbar_arrive_expect_tx(&bars->v_full[s], C::kTileBytes);
           for (int c = 0; c < C::kSub; ++c)
             tma_load_4d(smem + C::kOffV + s * C::kTileBytes + c * C::kSubBytes, &tmV, &bars->v_full[s], c * 64,
-                        j * kBN, h, b);
+                        (kbase + j) * kBN, hk, b);
         }
       }
     } else if (warp == 9) {
@@ -327,15 +342,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           umma_commit(&bars->o_done[t]);
         };
+        // Stream tile j is key tile kbase + j; for query tile t it is local
+        // tile j - (klo[t] - kbase), active when that lies in [0, nkt[t]).
+        auto local = [&](int t, int j) { return j - (klo[t] - kbase); };
+        auto active = [&](int t, int j) { return local(t, j) >= 0 && local(t, j) < nkt[t]; };
         // Issue order: S_0(0) S_1(0) | PV_0(j) S_0(j+1) PV_1(j) S_1(j+1) | ...
         // S_t(j+1) overwrites the columns PV_t(j) reads P_t(j) from; the tensor
         // pipe executes one thread's MMAs in issue order, so PV_t(j) has read
-        // P_t(j) before S_t(j+1) writes there.
+        // P_t(j) before S_t(j+1) writes there.  A query tile whose first key
+        // tile is a later stream tile gets its first S in the iteration before.
         bool ok = wait_bar(&bars->q_full, 0, w, 3) && wait_bar(&bars->k_full[0], 0, w, 4);
         if (ok) {
           tc_fence_after();
           for (int t = 0; t < 2; ++t)
-            if (nkt[t] > 0) issue_s(t, 0);
+            if (active(t, 0)) issue_s(t, 0);
           umma_commit(&bars->k_empty[0]);
         }
         for (int j = 0; ok && j < nk; ++j) {
@@ -344,11 +364,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!(ok = wait_bar(&bars->v_full[s], (j / C::kStages) & 1, w, 6))) break;
           bool next_k = false;
           for (int t = 0; t < 2; ++t) {
-            if (j >= nkt[t]) continue;
-            if (!(ok = wait_bar(&bars->p_full[t], j & 1, w, 7))) break;
-            tc_fence_after();
-            issue_pv(t, s, j > 0);
-            if (j + 1 < nkt[t]) {
+            if (active(t, j)) {
+              const int jl = local(t, j);
+              if (!(ok = wait_bar(&bars->p_full[t], jl & 1, w, 7))) break;
+              tc_fence_after();
+              issue_pv(t, s, jl > 0);
+            }
+            if (j + 1 < nk && active(t, j + 1)) {
               if (!next_k) {
                 if (!(ok = wait_bar(&bars->k_full[sn], ((j + 1) / C::kStages) & 1, w, 5))) break;
                 tc_fence_after();

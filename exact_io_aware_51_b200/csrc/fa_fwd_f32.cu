@@ -30,6 +30,7 @@ __global__ void __launch_bounds__(kRows * (D / 64))
 
   const int h = blockIdx.y;
   const int b = blockIdx.z;
+  const int hk = h / (a.H / a.Hkv);  // K/V head of this query head
   const int row0 = blockIdx.x * kRows;
   const int tid = threadIdx.x;
   const int part = tid % TPR;
@@ -49,15 +50,17 @@ __global__ void __launch_bounds__(kRows * (D / 64))
   }
   float m = -INFINITY, l = 0.f;
 
-  const int last_key = a.causal ? min(a.N, row0 + kRows) : a.N;  // keys [0, last_key)
-  for (int k0 = 0; k0 < last_key; k0 += kKT) {
+  // keys some row of this CTA may see: [first_key, last_key)
+  const int first_key = max(0, row0 - a.wl) / kKT * kKT;
+  const int last_key = min(a.N - 1, row0 + kRows - 1 + a.wr) + 1;
+  for (int k0 = first_key; k0 < last_key; k0 += kKT) {
     __syncthreads();
     for (int e = tid * 4; e < kKT * D; e += kThreads * 4) {
       const int kr = e / D, kc = e % D;
       const int key = k0 + kr;
       float4 kx = make_float4(0.f, 0.f, 0.f, 0.f), vx = kx;
       if (key < a.N) {
-        const size_t off = ((static_cast<size_t>(b) * a.N + key) * a.H + h) * D + kc;
+        const size_t off = ((static_cast<size_t>(b) * a.N + key) * a.Hkv + hk) * D + kc;
         kx = *reinterpret_cast<const float4*>(K + off);
         vx = *reinterpret_cast<const float4*>(V + off);
       }
@@ -75,7 +78,7 @@ __global__ void __launch_bounds__(kRows * (D / 64))
       for (int i = 0; i < 64; ++i) dot = fmaf(q[i], sK[jj][part * 64 + i], dot);
       if (TPR == 2) dot += __shfl_xor_sync(0xffffffffu, dot, 1);
       const int key = k0 + jj;
-      const bool visible = key < a.N && (!a.causal || key <= qrow);
+      const bool visible = key < a.N && key <= qrow + a.wr && key >= qrow - a.wl;
       s[jj] = visible ? dot : -INFINITY;
       mx = fmaxf(mx, s[jj]);
     }

@@ -18,19 +18,28 @@ struct DevCtl {
   int inject;                   // test-only fault injection (0 = off)
 };
 
+// Visibility mask of every pass: key k is visible to query q when
+// q - wl <= k <= q + wr and k < N (wl, wr >= 0; a value >= N leaves that side
+// unbounded).  (wl, wr) = (N, N) is unmasked attention, (N, 0) causal, and a
+// finite wl a sliding window.  `causal` is set exactly for (N, 0); it only
+// selects the order in which CTAs take their tiles.
 struct FwdArgs {
   int B, H, N, d;
+  int Hkv;           // K/V heads; query head h reads K/V head h / (H / Hkv)
   float scale_log2;  // softmax scale * log2(e)
   int causal;
+  int wl, wr;        // window (see above)
   void* O;           // [B, N, H, d]
   float* LSE;        // [B, H, N], natural log
 };
 
 struct BwdArgs {
   int B, H, N, d, Npad;
+  int Hkv;           // K/V heads (dK, dV are [B, N, Hkv, d])
   float scale;       // softmax scale
   float scale_log2;  // scale * log2(e)
   int causal;
+  int wl, wr;        // window (see FwdArgs)
   const void* O;
   const void* dO;
   const float* LSE;  // [B, H, N] natural log

@@ -83,6 +83,34 @@ int fa_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, int
            float scale, int causal, int dtype, void* stream);
 
 /*
+ * Forward pass with grouped-query attention ("Flash Attention"
+ * (karlkratz.de), "Grouped Query Attention"): Hkv key/value heads, each
+ * shared by H / Hkv consecutive query heads; query head h attends with K/V
+ * head h / (H / Hkv).  Hkv = H is fa_fwd; Hkv = 1 is multi-query attention.
+ *   Q, O     [B, N, H, d];  K, V  [B, N, Hkv, d];  LSE  [B, H, N].
+ *   Hkv      1 <= Hkv <= H and H % Hkv == 0 (FA_ERR_INVALID_ARG otherwise;
+ *            Hkv = 0 only with H = 0).
+ * Other arguments, results and errors as fa_fwd.
+ */
+int fa_fwd_gqa(const void* Q, const void* K, const void* V, void* O, float* LSE, int B, int H, int Hkv, int N,
+               int d, float scale, int causal, int dtype, void* stream);
+
+/*
+ * Forward pass with a sliding-window mask ("Flash Attention" (karlkratz.de),
+ * "Sliding Window Attention": each position attends to a fixed neighbourhood,
+ * and blocks outside the window are neither loaded nor computed).
+ *   Key j is visible to query i when
+ *     i - window_left <= j <= i + window_right   (and j < N);
+ *   a bound of -1 leaves that side open.  (-1, -1) is fa_fwd_gqa without the
+ *   causal mask, (-1, 0) with it; a window of W tokens ending at the query
+ *   (Mistral-style) is (W - 1, 0).  Bounds below -1 are FA_ERR_INVALID_ARG.
+ *   Every row sees at least its own key, so no row is empty.
+ * Other arguments (grouped K/V heads included), results and errors as fa_fwd_gqa.
+ */
+int fa_fwd_window(const void* Q, const void* K, const void* V, void* O, float* LSE, int B, int H, int Hkv, int N,
+                  int d, float scale, int window_left, int window_right, int dtype, void* stream);
+
+/*
  * Bytes of device workspace fa_bwd needs for this problem: an fp32 dQ
  * accumulator [B, N, H, d] plus two fp32 [B, H, roundup(N, 128)] rows
  * (rowsum(dO * O) and LSE * log2 e), each region 256-byte aligned.  This is
@@ -103,11 +131,37 @@ size_t fa_bwd_workspace_size(int B, int H, int N, int d, int dtype);
  *   workspace       device buffer of at least fa_bwd_workspace_size() bytes,
  *                   256-byte aligned; overwritten.
  * Currently dtype FA_BF16 with d = 128 (FA_ERR_UNSUPPORTED otherwise).
- * dQ is accumulated with fp32 atomics, so it is not bitwise deterministic.
+ * dQ is summed over key tiles by fp32 reduce-adds in L2 whose order varies
+ * from run to run, so it is not bitwise deterministic.
  */
 int fa_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO, const float* LSE, void* dQ,
            void* dK, void* dV, int B, int H, int N, int d, float scale, int causal, int dtype, void* workspace,
            size_t workspace_bytes, void* stream);
+
+/*
+ * Backward pass with grouped-query attention (see fa_fwd_gqa).  The gradient
+ * of a shared K/V head is the sum over its H / Hkv query heads:
+ *   dK[:, :, g] = sum over h in group g of scale * dS_h^T Q_h,
+ *   dV[:, :, g] = sum over h in group g of P_h^T dO_h,
+ * accumulated in fp32 inside one CTA per (key tile, K/V head) and written once.
+ *   Q, O, dO, dQ  [B, N, H, d];  K, V, dK, dV  [B, N, Hkv, d];  LSE  [B, H, N].
+ *   workspace     as fa_bwd: fa_bwd_workspace_size(B, H, N, d, dtype) bytes
+ *                 (it depends on the query heads only).
+ * Other arguments, results and errors as fa_bwd.
+ */
+int fa_bwd_gqa(const void* Q, const void* K, const void* V, const void* O, const void* dO, const float* LSE,
+               void* dQ, void* dK, void* dV, int B, int H, int Hkv, int N, int d, float scale, int causal, int dtype,
+               void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Backward pass under the sliding-window mask of fa_fwd_window (same
+ * window_left / window_right meaning); the forward's O and LSE must come from
+ * the same window.  Each key tile visits only the query tiles inside its
+ * window.  Other arguments, results and errors as fa_bwd_gqa.
+ */
+int fa_bwd_window(const void* Q, const void* K, const void* V, const void* O, const void* dO, const float* LSE,
+                  void* dQ, void* dK, void* dV, int B, int H, int Hkv, int N, int d, float scale, int window_left,
+                  int window_right, int dtype, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * fa_bwd for callers that cannot allocate device memory when they run the

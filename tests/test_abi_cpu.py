@@ -110,3 +110,65 @@ def test_python_binding_refuses_cpu_tensors(L):
     q = torch.zeros(1, 128, 1, 64, dtype=torch.bfloat16)
     with pytest.raises(ValueError, match="CUDA"):
         fa.fwd(q, q, q)
+
+
+def test_gqa_head_count_validation(L):
+    """fa_fwd_gqa / fa_bwd_gqa: Hkv must divide H (grouped-query attention, "Flash Attention"
+    (karlkratz.de), "Grouped Query Attention"); checked before any device work."""
+    f = L.fa_fwd_gqa
+    for H, Hkv in ((8, 3), (8, 0), (8, 16), (8, -1)):
+        assert f(16, 16, 16, 16, 16, 1, H, Hkv, 128, 64, 0.125, 0, 0, None) == -1, (H, Hkv)
+    # valid groupings get past the head check to the next one (a misaligned pointer)
+    for H, Hkv in ((8, 1), (8, 2), (8, 8), (64, 8)):
+        assert f(8, 16, 16, 16, 16, 1, H, Hkv, 128, 64, 0.125, 0, 0, None) == -3, (H, Hkv)
+    # empty problems stay no-ops
+    assert f(None, None, None, None, None, 1, 0, 0, 128, 64, 0.125, 0, 0, None) == 0
+    b = L.fa_bwd_gqa
+    args = [16] * 9
+    ws = L.fa_bwd_workspace_size(1, 8, 128, 128, 0)
+    assert b(*args, 1, 8, 3, 128, 128, 0.1, 0, 0, 256, ws, None) == -1
+    assert b(*args, 1, 8, 0, 128, 128, 0.1, 0, 0, 256, ws, None) == -1
+    bad = list(args)
+    bad[7] = 24  # misaligned dK: the head check passed
+    assert b(*bad, 1, 8, 2, 128, 128, 0.1, 0, 0, 256, ws, None) == -3
+
+
+def test_python_binding_checks_gqa_shapes(L):
+    import torch
+    q = torch.zeros(1, 128, 8, 64, dtype=torch.bfloat16)
+    k = torch.zeros(1, 128, 3, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="Hkv dividing"):
+        fa.fwd(q, k, k)
+    k2 = torch.zeros(1, 128, 2, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="Hkv dividing"):
+        fa.fwd(q, k2[:, :64], k2[:, :64])
+    with pytest.raises(ValueError, match="share one shape"):
+        fa.fwd(q, k2, k2[:, :, :1])
+    with pytest.raises(ValueError, match="CUDA"):
+        fa.fwd(q, k2, k2)  # a valid grouping reaches the device check
+
+
+def test_window_bound_validation(L):
+    """fa_fwd_window / fa_bwd_window: each bound is -1 (open) or >= 0, checked before device work."""
+    f = L.fa_fwd_window
+    for wl, wr in ((-2, 0), (0, -2), (-5, -5)):
+        assert f(16, 16, 16, 16, 16, 1, 2, 2, 128, 64, 0.125, wl, wr, 0, None) == -1, (wl, wr)
+    for wl, wr in ((-1, -1), (-1, 0), (0, 0), (4095, 0), (3, 7), (1 << 30, 1 << 30)):
+        assert f(8, 16, 16, 16, 16, 1, 2, 2, 128, 64, 0.125, wl, wr, 0, None) == -3, (wl, wr)
+    b = L.fa_bwd_window
+    args = [16] * 9
+    ws = L.fa_bwd_workspace_size(1, 2, 128, 128, 0)
+    assert b(*args, 1, 2, 2, 128, 128, 0.1, -2, 0, 0, 256, ws, None) == -1
+    bad = list(args)
+    bad[7] = 24
+    assert b(*bad, 1, 2, 2, 128, 128, 0.1, 64, 0, 0, 256, ws, None) == -3
+
+
+def test_python_window_bounds():
+    assert fa._window_bounds(False, (None, None)) == (-1, -1)
+    assert fa._window_bounds(True, (None, None)) == (-1, 0)
+    assert fa._window_bounds(True, (4095, None)) == (4095, 0)
+    assert fa._window_bounds(True, (10, 5)) == (10, 0)
+    assert fa._window_bounds(False, (3, 7)) == (3, 7)
+    with pytest.raises(ValueError):
+        fa._window_bounds(False, (-1, 0))
