@@ -19,8 +19,8 @@ import pathlib
 import torch
 
 __all__ = [
-    "FAError", "FA_BF16", "FA_FP32", "lib", "lib_path", "fwd", "bwd", "bwd_workspace_size",
-    "last_device_status", "set_wait_limit_ms", "debug_inject", "debug_umma", "status_string",
+    "FAError", "FA_BF16", "FA_FP32", "lib", "lib_path", "fwd", "fwd_fp8", "bwd", "bwd_workspace_size",
+    "last_device_status", "set_wait_limit_ms", "debug_inject", "debug_umma", "debug_umma_f8", "status_string",
     "set_kernel_events",
     "attention", "EXPORTED",
 ]
@@ -34,7 +34,7 @@ _LIB = None
 EXPORTED = ("fa_fwd", "fa_bwd_workspace_size", "fa_bwd", "fa_status_string", "fa_last_cuda_error",
             "fa_last_device_status", "fa_set_wait_limit_ms", "fa_debug_inject", "fa_debug_umma",
             "fa_version", "fa_set_kernel_events", "fa_bwd_static_scratch", "fa_fwd_gqa", "fa_bwd_gqa",
-            "fa_fwd_window", "fa_bwd_window")
+            "fa_fwd_window", "fa_bwd_window", "fa_debug_umma_f8", "fa_fwd_fp8")
 
 
 class FAError(RuntimeError):
@@ -72,6 +72,8 @@ def lib() -> ctypes.CDLL:
     L.fa_fwd_gqa.restype = i
     L.fa_bwd_gqa.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp, sz, vp]
     L.fa_bwd_gqa.restype = i
+    L.fa_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, f, f, f, i, i, vp]
+    L.fa_fwd_fp8.restype = i
     L.fa_fwd_window.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, i, vp]
     L.fa_fwd_window.restype = i
     L.fa_bwd_window.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, i, vp, sz, vp]
@@ -88,6 +90,8 @@ def lib() -> ctypes.CDLL:
     L.fa_debug_inject.restype = None
     L.fa_debug_umma.argtypes = [vp, vp, vp, i, i, i, i, i, vp]
     L.fa_debug_umma.restype = i
+    L.fa_debug_umma_f8.argtypes = [vp, vp, vp, i, i, i, vp]
+    L.fa_debug_umma_f8.restype = i
     L.fa_bwd_static_scratch.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, i, vp]
     L.fa_bwd_static_scratch.restype = i
     L.fa_set_kernel_events.argtypes = [vp, vp]
@@ -176,6 +180,26 @@ def fwd(q, k, v, causal: bool = False, scale: float | None = None, out=None, lse
     return o, l
 
 
+def fwd_fp8(q, k, v, scale_q: float, scale_k: float, scale_v: float, causal: bool = False,
+            scale: float | None = None, window=None, out=None, lse=None, stream=None):
+    """Forward with 8-bit inputs: q [B, N, H, 128], k, v [B, N, Hkv, 128] as torch.float8_e4m3fn
+    (or their uint8 codes), each dequantised by its scale; returns (o bf16, lse fp32)."""
+    for t in (q, k, v):
+        if t.dtype not in (torch.float8_e4m3fn, torch.uint8):
+            raise TypeError("fwd_fp8 takes torch.float8_e4m3fn (or uint8 e4m3 codes)")
+    Hkv = _check_inputs(q, k, v)
+    B, N, H, d = q.shape
+    o = torch.empty((B, N, H, d), dtype=torch.bfloat16, device=q.device) if out is None else out
+    l = torch.empty((B, H, N), dtype=torch.float32, device=q.device) if lse is None else lse
+    wl, wr = _window_bounds(causal, (None, None) if window is None else window)
+    rc = lib().fa_fwd_fp8(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), l.data_ptr(), B, H, Hkv, N, d,
+                          _scale(scale, d), float(scale_q), float(scale_k), float(scale_v), wl, wr,
+                          _stream_handle(stream, q.device))
+    if rc != 0:
+        raise FAError(rc, "fa_fwd_fp8")
+    return o, l
+
+
 def bwd_workspace_size(B: int, H: int, N: int, d: int, dtype: int = FA_BF16) -> int:
     return int(lib().fa_bwd_workspace_size(B, H, N, d, dtype))
 
@@ -245,6 +269,17 @@ def debug_umma(a: torch.Tensor, b: torch.Tensor, a_mn_major: int, b_mn_major: in
                              int(b_mn_major), int(a_tmem), _stream_handle(stream, a.device))
     if rc != 0:
         raise FAError(rc, "fa_debug_umma")
+    return dmat
+
+
+def debug_umma_f8(a: torch.Tensor, b: torch.Tensor, b_mn_major: int, a_tmem: int = 0, stream=None) -> torch.Tensor:
+    """One 8-bit tcgen05 MMA tile D = A B^T (test-only): a [128, 128], b [N, 128] e4m3 (uint8 bytes) cuda."""
+    n = b.shape[0]
+    dmat = torch.empty((128, n), dtype=torch.float32, device=a.device)
+    rc = lib().fa_debug_umma_f8(a.data_ptr(), b.data_ptr(), dmat.data_ptr(), n, int(b_mn_major), int(a_tmem),
+                                _stream_handle(stream, a.device))
+    if rc != 0:
+        raise FAError(rc, "fa_debug_umma_f8")
     return dmat
 
 

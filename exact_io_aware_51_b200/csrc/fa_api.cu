@@ -198,6 +198,19 @@ CUresult make_tile_map(CUtensorMap* map, const void* base, int B, int N, int H, 
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
 }
 
+CUresult make_tile_map_e4m3(CUtensorMap* map, const void* base, int B, int N, int H, int d, int rows) {
+  if (!encoder()) return CUDA_ERROR_NOT_FOUND;
+  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(H),
+                              static_cast<cuuint64_t>(B)};
+  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(H) * d, static_cast<cuuint64_t>(d),
+                                 static_cast<cuuint64_t>(N) * H * d};
+  const cuuint32_t box[4] = {128u, static_cast<cuuint32_t>(rows), 1u, 1u};
+  const cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+  return g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+}
+
 CUresult make_dq_accum_map(CUtensorMap* map, float* base, int B, int N, int H, int d) {
   if (!encoder()) return CUDA_ERROR_NOT_FOUND;
   const cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(H),
@@ -314,6 +327,47 @@ int fa_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, int
   return fa_fwd_window(Q, K, V, O, LSE, B, H, H, N, d, scale, -1, causal ? 0 : -1, dtype, stream);
 }
 
+int fa_fwd_fp8(const void* Q, const void* K, const void* V, void* O, float* LSE, int B, int H, int Hkv, int N, int d,
+               float scale, float scale_q, float scale_k, float scale_v, int window_left, int window_right,
+               void* stream) {
+  int rc = check_shape(B, H, N, d, FA_BF16);
+  if (rc) return rc;
+  if (d != 128) return FA_ERR_UNSUPPORTED;
+  if ((rc = check_kv_heads(H, Hkv))) return rc;
+  if ((rc = check_window(window_left, window_right))) return rc;
+  if ((rc = check_scale(scale)) || (rc = check_scale(scale_q)) || (rc = check_scale(scale_k)) ||
+      (rc = check_scale(scale_v)))
+    return rc;
+  if (static_cast<long long>(B) * H * N == 0) return FA_OK;
+  if (!Q || !K || !V || !O || !LSE) return FA_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(LSE)) return FA_ERR_MISALIGNED;
+  DeviceState* st = nullptr;
+  if ((rc = device_state(&st))) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  FwdArgs a;
+  a.B = B;
+  a.H = H;
+  a.Hkv = Hkv;
+  a.N = N;
+  a.d = d;
+  // the per-tensor scales of Q and K fold into the softmax's exponent scale
+  a.scale_log2 = static_cast<float>(static_cast<double>(scale) * scale_q * scale_k * 1.4426950408889634);
+  set_window(window_left, window_right, &a.wl, &a.wr, &a.causal);
+  a.O = O;
+  a.LSE = LSE;
+  CUtensorMap tq, tk, tv;
+  CUresult r;
+  if ((r = make_tile_map_e4m3(&tq, Q, B, N, H, d, 128)) != CUDA_SUCCESS ||
+      (r = make_tile_map_e4m3(&tk, K, B, N, Hkv, d, 128)) != CUDA_SUCCESS ||
+      (r = make_tile_map_e4m3(&tv, V, B, N, Hkv, d, 128)) != CUDA_SUCCESS)
+    return fail_encode(r);
+  if (t_ev_start) cudaEventRecord(t_ev_start, s);
+  cudaError_t e = launch_fwd_fp8(tq, tk, tv, a, scale_v, make_ctl(*st), s);
+  if (e != cudaSuccess) return fail_cuda(e);
+  if (t_ev_stop) cudaEventRecord(t_ev_stop, s);
+  return FA_OK;
+}
+
 size_t fa_bwd_workspace_size(int B, int H, int N, int d, int dtype) {
   if (check_shape(B, H, N, d, dtype) != FA_OK) return 0;
   if (static_cast<long long>(B) * H * N == 0) return 0;
@@ -409,6 +463,18 @@ int fa_debug_umma(const void* A, const void* B, float* D, int N, int K, int a_mn
   if (rc) return rc;
   cudaError_t e = launch_umma_probe(A, B, D, N, K, a_mn_major ? 1 : 0, b_mn_major ? 1 : 0, a_tmem ? 1 : 0,
                                     static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail_cuda(e);
+  return FA_OK;
+}
+
+int fa_debug_umma_f8(const void* A, const void* B, float* D, int N, int b_mn_major, int a_tmem, void* stream) {
+  if (!A || !B || !D) return FA_ERR_INVALID_ARG;
+  if (N != 64 && N != 128) return FA_ERR_UNSUPPORTED;
+  DeviceState* st = nullptr;
+  int rc = device_state(&st);
+  if (rc) return rc;
+  cudaError_t e =
+      launch_umma_probe_f8(A, B, D, N, b_mn_major ? 1 : 0, a_tmem ? 1 : 0, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return fail_cuda(e);
   return FA_OK;
 }

@@ -55,6 +55,10 @@ struct BwdArgs {
 // positions x 64 features of one (b, h); 128-byte swizzle.
 CUresult make_tile_map(CUtensorMap* map, const void* base, int B, int N, int H, int d, int rows);
 
+// TMA descriptor for a [B, N, H, d] e4m3 (byte) tensor with d = 128: a box of
+// `rows` sequence positions x 128 features of one (b, h), 128-byte swizzle.
+CUresult make_tile_map_e4m3(CUtensorMap* map, const void* base, int B, int N, int H, int d, int rows);
+
 // TMA descriptor for the fp32 [B, N, H, d] dQ accumulator with a box of 64
 // sequence positions x d features of one (b, h), no swizzle (for TMA reduce-add).
 CUresult make_dq_accum_map(CUtensorMap* map, float* base, int B, int N, int H, int d);
@@ -62,6 +66,8 @@ CUresult make_dq_accum_map(CUtensorMap* map, float* base, int B, int N, int H, i
 // Kernel launchers (each returns the cudaError_t of the launch).
 cudaError_t launch_fwd_bf16(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const FwdArgs& a, const DevCtl& c, cudaStream_t s);
+cudaError_t launch_fwd_fp8(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const FwdArgs& a,
+                           float out_scale, const DevCtl& c, cudaStream_t s);
 cudaError_t launch_fwd_f32(const float* Q, const float* K, const float* V, const FwdArgs& a, cudaStream_t s);
 cudaError_t launch_bwd_pre(const BwdArgs& a, cudaStream_t s);
 cudaError_t launch_bwd_main(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
@@ -72,5 +78,7 @@ cudaError_t launch_bwd_dq(const BwdArgs& a, cudaStream_t s);
 // Test-only single-tile MMA probe (see fa_debug_umma in the public header).
 cudaError_t launch_umma_probe(const void* A, const void* B, float* D, int N, int K, int a_mn_major,
                               int b_mn_major, int a_tmem, cudaStream_t s);
+cudaError_t launch_umma_probe_f8(const void* A, const void* B, float* D, int N, int b_mn_major, int a_tmem,
+                                 cudaStream_t s);
 
 }  // namespace fa

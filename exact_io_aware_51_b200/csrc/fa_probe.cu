@@ -116,7 +116,109 @@ __global__ void __launch_bounds__(128, 1)
   }
 }
 
+// The same probe for the 8-bit (e4m3) MMA with K = 128: A [128][128] K-major in
+// shared memory or in TMEM (four elements per column), B [N][128] K-major or
+// stored MN-major ([128 k][N], N contiguous).  One 128-byte swizzled row holds
+// all 128 elements of a K-major row.
+__global__ void __launch_bounds__(128, 1)
+    umma_probe_f8_kernel(const uint8_t* __restrict__ A, const uint8_t* __restrict__ B, float* __restrict__ D, int N,
+                         int b_mn, int a_tmem) {
+  constexpr int K = 128;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;          // 128 x 128 bytes
+  uint8_t* sB = smem + 16384;  // N x 128 bytes (N <= 128)
+  __shared__ uint64_t bar;
+  __shared__ uint32_t tbase;
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+
+  for (int e = tid; e < 128 * K; e += 128) {
+    const int m = e / K, k = e % K;
+    sA[sw128_offset(m, k / 16) + (k % 16)] = A[e];
+  }
+  for (int e = tid; e < N * K; e += 128) {
+    const int n = e / K, k = e % K;
+    const uint32_t off = (b_mn == 0) ? sw128_offset(n, k / 16) + (k % 16) : sw128_offset(k, n / 16) + (n % 16);
+    sB[off] = B[e];
+  }
+  if (tid == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) tmem_alloc(&tbase, 512);
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tbase;
+  const uint32_t lane_bits = static_cast<uint32_t>(warp * 32) << 16;
+
+  if (a_tmem) {
+    // row m = tid into lane m; column 256 + c holds k = 4c .. 4c + 3 (k = 4c in the low byte)
+    for (int c0 = 0; c0 < K / 4; c0 += 16) {
+      uint32_t r[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const uint8_t* a4 = A + tid * K + 4 * (c0 + i);
+        r[i] = static_cast<uint32_t>(a4[0]) | (static_cast<uint32_t>(a4[1]) << 8) |
+               (static_cast<uint32_t>(a4[2]) << 16) | (static_cast<uint32_t>(a4[3]) << 24);
+      }
+      tmem_st16(tmem + lane_bits + 256 + c0, r);
+    }
+    tmem_wait_st();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+  }
+
+  if (tid == 0) {
+    const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sB);
+    const uint32_t idesc = idesc_e4m3(128, N, 0, b_mn);
+    for (int kk = 0; kk < K / 32; ++kk) {
+      const uint64_t bd = (b_mn == 0) ? sw128_desc(b0 + kk * 32, 16, 1024) : sw128_desc(b0 + kk * 4096, 16384, 1024);
+      if (a_tmem)
+        umma_ts_f8(tmem, tmem + 256 + kk * 8, bd, idesc, kk > 0 ? 1u : 0u);
+      else
+        umma_ss_f8(tmem, sw128_desc(a0 + kk * 32, 16, 1024), bd, idesc, kk > 0 ? 1u : 0u);
+    }
+    umma_commit(&bar);
+  }
+  const uint64_t t0 = globaltimer_ns();
+  bool done = false;
+  while (!(done = mbar_try_wait(&bar, 0)) && globaltimer_ns() - t0 < 2000000000ull) {
+  }
+  done = __all_sync(0xffffffffu, done);
+  tc_fence_after();
+  if (done) {
+    for (int c0 = 0; c0 < N; c0 += 32) {
+      uint32_t r[32];
+      tmem_ld32(tmem + lane_bits + c0, r);
+      tmem_wait_ld();
+      reg_fence32(r);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) D[tid * N + c0 + i] = __uint_as_float(r[i]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_umma_probe_f8(const void* A, const void* B, float* D, int N, int b_mn, int a_tmem,
+                                 cudaStream_t s) {
+  constexpr int smem = 32768 + 1024;
+  cudaError_t e = cudaFuncSetAttribute(umma_probe_f8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  umma_probe_f8_kernel<<<1, 128, smem, s>>>(static_cast<const uint8_t*>(A), static_cast<const uint8_t*>(B), D, N,
+                                            b_mn, a_tmem);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_umma_probe(const void* A, const void* B, float* D, int N, int K, int a_mn, int b_mn, int a_tmem,
                               cudaStream_t s) {

@@ -111,6 +111,25 @@ int fa_fwd_window(const void* Q, const void* K, const void* V, void* O, float* L
                   int d, float scale, int window_left, int window_right, int dtype, void* stream);
 
 /*
+ * Forward pass with 8-bit inputs (FP8 attention as FlashAttention-3 runs it:
+ * "Flash Attention" (karlkratz.de), "Versionen").
+ *   Q        [B, N, H, d] e4m3 codes (one byte each); the value is scale_q * code.
+ *   K, V     [B, N, Hkv, d] e4m3 codes with scales scale_k, scale_v.
+ *   O        [B, N, H, d] bf16 output; LSE [B, H, N] fp32 natural log.
+ *   scale    softmax scale (finite, > 0); scale_q, scale_k, scale_v finite, > 0.
+ *   Hkv, window_left, window_right as fa_fwd_window (-1, -1: no mask; -1, 0: causal).
+ *   d        128 only (FA_ERR_UNSUPPORTED otherwise).
+ * S = Q K^T accumulates the 8-bit products in fp32 on the tensor cores; the
+ * probabilities are rounded to e4m3 (after scaling by 2^4, so the largest is at
+ * most 256) before P V, and the row sums use the unrounded fp32 values.  The
+ * result is the exact attention of the dequantised inputs up to those
+ * roundings (see the design notes for the bound the tests use).
+ */
+int fa_fwd_fp8(const void* Q, const void* K, const void* V, void* O, float* LSE, int B, int H, int Hkv, int N,
+               int d, float scale, float scale_q, float scale_k, float scale_v, int window_left, int window_right,
+               void* stream);
+
+/*
  * Bytes of device workspace fa_bwd needs for this problem: an fp32 dQ
  * accumulator [B, N, H, d] plus two fp32 [B, H, roundup(N, 128)] rows
  * (rowsum(dO * O) and LSE * log2 e), each region 256-byte aligned.  This is
@@ -231,6 +250,15 @@ void fa_set_kernel_events(void* start, void* stop);
  */
 int fa_debug_umma(const void* A, const void* B, float* D, int N, int K, int a_mn_major, int b_mn_major,
                   int a_tmem, void* stream);
+
+/*
+ * Test-only: the same probe for the 8-bit MMA (kind::f8f6f4, e4m3 operands,
+ * fp32 accumulation) with K = 128: A [128][128] and B [N][128] e4m3 bytes
+ * (row-major device arrays), D [128][N] fp32.  b_mn_major stores B with N
+ * contiguous; a_tmem reads A from tensor memory (four elements per column).
+ * N must be 64 or 128.
+ */
+int fa_debug_umma_f8(const void* A, const void* B, float* D, int N, int b_mn_major, int a_tmem, void* stream);
 
 /* Library version: major * 10000 + minor * 100 + patch. */
 int fa_version(void);

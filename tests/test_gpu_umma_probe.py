@@ -41,3 +41,24 @@ def test_umma_tile(n, k, a_mn, b_mn, a_tmem):
     torch.cuda.synchronize()
     ref = a.double().numpy() @ b.double().numpy().T
     assert rel_err(d.cpu(), ref) < 1e-5
+
+
+# 8-bit MMA (e4m3, K = 128): S = Q K^T (both K-major), O += P V with P in TMEM and
+# V stored [keys][d] (B MN-major), and MN-major B from shared memory.
+F8_CASES = [(128, 0, 0), (64, 0, 0), (128, 1, 1), (128, 1, 0), (64, 1, 1)]
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("n,b_mn,a_tmem", F8_CASES)
+def test_umma_tile_e4m3(n, b_mn, a_tmem):
+    need_gpu()
+    g = torch.Generator().manual_seed(n * 10 + b_mn * 2 + a_tmem)
+    a = (torch.randn(128, 128, generator=g) * 4).to(torch.float8_e4m3fn)
+    b = (torch.randn(n, 128, generator=g) * 4).to(torch.float8_e4m3fn)
+    d = fa.debug_umma_f8(a.view(torch.uint8).cuda(), b.view(torch.uint8).cuda(), b_mn, a_tmem)
+    torch.cuda.synchronize()
+    # e4m3 values and their products are exact; the tensor core's fp32 accumulation
+    # of 8-bit products may keep fewer mantissa bits than an fp32 add, so the
+    # bound is 1e-3 (a wrong operand layout gives errors of order 1)
+    ref = a.double().numpy() @ b.double().numpy().T
+    assert rel_err(d.cpu(), ref) < 1e-3
