@@ -172,3 +172,19 @@ def test_python_window_bounds():
     assert fa._window_bounds(False, (3, 7)) == (3, 7)
     with pytest.raises(ValueError):
         fa._window_bounds(False, (-1, 0))
+
+
+def test_fp8_forward_validation(L):
+    """fa_fwd_fp8 refuses what it does not implement before touching the device."""
+    f = L.fa_fwd_fp8
+    ok = (1.0, 1.0, 1.0)
+    # d other than 128
+    assert f(16, 16, 16, 16, 16, 1, 2, 2, 128, 64, 0.1, *ok, -1, -1, None) == -2
+    # bad scales (softmax scale and each tensor scale)
+    for bad in ((0.0, 1.0, 1.0, 1.0), (0.1, -1.0, 1.0, 1.0), (0.1, 1.0, float("nan"), 1.0), (0.1, 1.0, 1.0, 0.0)):
+        assert f(16, 16, 16, 16, 16, 1, 2, 2, 128, 128, *bad, -1, -1, None) == -1, bad
+    # grouping and window checks, then alignment
+    assert f(16, 16, 16, 16, 16, 1, 4, 3, 128, 128, 0.1, *ok, -1, -1, None) == -1
+    assert f(16, 16, 16, 16, 16, 1, 4, 2, 128, 128, 0.1, *ok, -3, -1, None) == -1
+    assert f(8, 16, 16, 16, 16, 1, 4, 2, 128, 128, 0.1, *ok, 64, 0, None) == -3
+    assert f(None, None, None, None, None, 0, 4, 2, 128, 128, 0.1, *ok, -1, -1, None) == 0
