@@ -52,6 +52,10 @@ Readings where the pages are silent (all recorded in the design notes):
   Attention") is a (left, right) pair: key j is visible to query i when
   i - left <= j <= i + right; the page's window of 4096 tokens is
   (4095, 0), the position and the 4095 before it.
+* a block-sparse mask ("Flash Attention" (Ultralytics glossary), "Flash
+  Attention и смежные понятия") is a 0/1 array over 128 x 128 blocks of the
+  score matrix (one per query head, or one shared); a row whose blocks are all
+  0 sees no key and gets O = 0, LSE = -inf.
 
 ``blocked_forward_head`` restates the pages' online-softmax algorithm (key
 blocks streamed, running row max and sum, rescale when the max grows) and is
@@ -84,7 +88,7 @@ def _f64(x) -> np.ndarray:
     return a.astype(np.float64, copy=False)
 
 
-def hidden_keys(rows, nk: int, causal: bool, window=None) -> np.ndarray:
+def hidden_keys(rows, nk: int, causal: bool, window=None, block_mask=None, block: int = 128) -> np.ndarray:
     """Boolean [len(rows), nk] mask: True where key j is hidden from query row i.
 
     Query row i sits at sequence position i (top-left alignment).
@@ -94,6 +98,12 @@ def hidden_keys(rows, nk: int, causal: bool, window=None) -> np.ndarray:
       (karlkratz.de), section "Sliding Window Attention": each position attends
       to a fixed neighbourhood; the page's 4096-token window is read as
       (left, right) = (4095, 0): the position itself and the 4095 before it.
+    * block_mask: a [ceil(Nq / block), ceil(nk / block)] array; key j is hidden
+      from row i when block_mask[i // block, j // block] is 0.  "Flash
+      Attention" (Ultralytics glossary), "Flash Attention и смежные понятия":
+      sparse attention scores only chosen query/key pairs, and the block-sparse
+      form skips the empty blocks.
+    The conditions combine: a key is visible only when every given one allows it.
     """
     rows = np.asarray(rows, dtype=np.int64)[:, None]
     cols = np.arange(nk)[None, :]
@@ -106,10 +116,13 @@ def hidden_keys(rows, nk: int, causal: bool, window=None) -> np.ndarray:
             hidden |= cols > rows + right
         if left is not None:
             hidden |= cols < rows - left
+    if block_mask is not None:
+        bm = np.asarray(block_mask) != 0
+        hidden |= ~bm[rows // block, cols // block]
     return hidden
 
 
-def scores_head(q, k, scale: float, causal: bool, window=None) -> np.ndarray:
+def scores_head(q, k, scale: float, causal: bool, window=None, block_mask=None) -> np.ndarray:
     """S = scale * Q K^T for one (batch, head), with the mask applied.
 
     q: [Nq, d], k: [Nk, d].  Masked entries are -inf (see ``hidden_keys`` for
@@ -120,8 +133,8 @@ def scores_head(q, k, scale: float, causal: bool, window=None) -> np.ndarray:
     q = _f64(q)
     k = _f64(k)
     s = float(scale) * (q @ k.T)
-    if causal or window is not None:
-        hidden = hidden_keys(np.arange(s.shape[0]), s.shape[1], causal, window)
+    if causal or window is not None or block_mask is not None:
+        hidden = hidden_keys(np.arange(s.shape[0]), s.shape[1], causal, window, block_mask)
         s = np.where(hidden, -np.inf, s)
     return s
 
@@ -143,7 +156,7 @@ def probs_head(s: np.ndarray):
     return p, lse
 
 
-def forward_head(q, k, v, scale: float, causal: bool, window=None):
+def forward_head(q, k, v, scale: float, causal: bool, window=None, block_mask=None):
     """O = softmax(scale Q K^T + mask) V and LSE for one (batch, head).
 
     q, k, v: [N, d].  Returns O [N, d] float64 and LSE [N] float64.
@@ -151,12 +164,12 @@ def forward_head(q, k, v, scale: float, causal: bool, window=None):
     "Flash Attention" (karlkratz.de), "Speicherbedarf und Laufzeitverhalten"
     (same result, not an approximation).
     """
-    s = scores_head(q, k, scale, causal, window)
+    s = scores_head(q, k, scale, causal, window, block_mask)
     p, lse = probs_head(s)
     return p @ _f64(v), lse
 
 
-def forward_rows_head(q, k, v, rows, scale: float, causal: bool, window=None):
+def forward_rows_head(q, k, v, rows, scale: float, causal: bool, window=None, block_mask=None):
     """Forward restricted to the query rows ``rows`` of one (batch, head).
 
     A row of O and its LSE depend only on that query row and all of K and V,
@@ -167,13 +180,13 @@ def forward_rows_head(q, k, v, rows, scale: float, causal: bool, window=None):
     q = _f64(q)
     k = _f64(k)
     s = float(scale) * (q[rows] @ k.T)
-    if causal or window is not None:
-        s = np.where(hidden_keys(rows, k.shape[0], causal, window), -np.inf, s)
+    if causal or window is not None or block_mask is not None:
+        s = np.where(hidden_keys(rows, k.shape[0], causal, window, block_mask), -np.inf, s)
     p, lse = probs_head(s)
     return p @ _f64(v), lse
 
 
-def backward_head(q, k, v, do, scale: float, causal: bool, window=None):
+def backward_head(q, k, v, do, scale: float, causal: bool, window=None, block_mask=None):
     """Gradients (dQ, dK, dV) of O = attention(Q, K, V) given dO, one head.
 
     Recomputes S and P from Q, K and V ("Flash Attention" (karlkratz.de),
@@ -184,7 +197,7 @@ def backward_head(q, k, v, do, scale: float, causal: bool, window=None):
     k = _f64(k)
     v = _f64(v)
     do = _f64(do)
-    s = scores_head(q, k, scale, causal, window)
+    s = scores_head(q, k, scale, causal, window, block_mask)
     p, _ = probs_head(s)
     o = p @ v
     dv = p.T @ do
@@ -264,7 +277,14 @@ def kv_head(h: int, n_heads: int, n_kv_heads: int) -> int:
     return h // (n_heads // n_kv_heads)
 
 
-def forward(Q, K, V, scale: float, causal: bool, heads=None, window=None):
+def _head_mask(block_mask, h):
+    if block_mask is None:
+        return None
+    bm = np.asarray(block_mask)
+    return bm[h] if bm.ndim == 3 else bm
+
+
+def forward(Q, K, V, scale: float, causal: bool, heads=None, window=None, block_mask=None):
     """Batched forward: Q [B, N, H, d]; K, V [B, N, Hkv, d] (numpy or CPU torch).
 
     Returns O [B, N, H, d] and LSE [B, H, N] in float64.  ``heads`` restricts
@@ -278,13 +298,13 @@ def forward(Q, K, V, scale: float, causal: bool, heads=None, window=None):
     LSE = np.full((b_, h_, n_), np.nan)
     for (b, h) in (heads if heads is not None else _all_heads(b_, h_)):
         g = kv_head(h, h_, hkv)
-        o, lse = forward_head(Q[b, :, h], K[b, :, g], V[b, :, g], scale, causal, window)
+        o, lse = forward_head(Q[b, :, h], K[b, :, g], V[b, :, g], scale, causal, window, _head_mask(block_mask, h))
         O[b, :, h] = o
         LSE[b, h] = lse
     return O, LSE
 
 
-def backward(Q, K, V, dO, scale: float, causal: bool, heads=None, window=None):
+def backward(Q, K, V, dO, scale: float, causal: bool, heads=None, window=None, block_mask=None):
     """Batched backward.  Returns dQ [B, N, H, d], dK and dV [B, N, Hkv, d] (float64).
 
     A K/V head shared by a group of query heads enters each of their
@@ -301,7 +321,8 @@ def backward(Q, K, V, dO, scale: float, causal: bool, heads=None, window=None):
     touched = set()
     for (b, h) in (heads if heads is not None else _all_heads(shape[0], shape[2])):
         g = kv_head(h, shape[2], hkv)
-        dq, dk, dv, _ = backward_head(Q[b, :, h], K[b, :, g], V[b, :, g], dO[b, :, h], scale, causal, window)
+        dq, dk, dv, _ = backward_head(Q[b, :, h], K[b, :, g], V[b, :, g], dO[b, :, h], scale, causal, window,
+                                      _head_mask(block_mask, h))
         dQ[b, :, h] = dq
         if (b, g) not in touched:
             touched.add((b, g))

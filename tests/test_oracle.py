@@ -289,6 +289,55 @@ def window_skipped_block_fraction(n, window, block, hidden=A.hidden_keys):
     return skipped / (nb * nb)
 
 
+BLOCK_MASKS = (
+    np.array([[1, 0, 1], [0, 1, 0], [1, 1, 1]]),
+    np.array([[0, 0, 1], [1, 0, 0], [0, 1, 1]]),
+    np.array([[1, 1, 1], [0, 0, 0], [1, 0, 1]]),   # middle row block sees nothing
+)
+
+
+def pin_blocksparse_rowwise(fwd=A.forward_head):
+    """Block-sparse mask over 128 x 128 blocks: each row is ordinary softmax
+    attention over the keys gathered from its visible blocks (no mask involved);
+    a row with no visible block gets O = 0 and LSE = -inf."""
+    n, d = 300, 4
+    q, k, v = 0.3 * _rand((n, d), 110), 0.3 * _rand((n, d), 111), _rand((n, 3), 112)
+    worst = 0.0
+    for bm in BLOCK_MASKS:
+        o, lse = fwd(q, k, v, 0.7, False, None, bm)
+        for i in range(n):
+            idx = np.concatenate([np.arange(128 * c, min(n, 128 * c + 128)) for c in range(3) if bm[i // 128, c]]
+                                 + [np.zeros(0, dtype=int)]).astype(int)
+            if idx.size == 0:
+                if not (np.all(o[i] == 0) and lse[i] == -np.inf):
+                    return math.inf
+                continue
+            s_ = 0.7 * (k[idx] @ q[i])
+            e = np.exp(s_ - s_.max())
+            worst = max(worst, float(np.max(np.abs(o[i] - e @ v[idx] / e.sum()))),
+                        abs(lse[i] - (s_.max() + math.log(e.sum()))))
+    return worst
+
+
+def pin_blocksparse_finite_differences(bwd=A.backward_head):
+    """Central differences of L = sum(dO * O) under a block mask, on sampled entries."""
+    n, d = 300, 3
+    q, k, v, do = (0.3 * _rand((n, d), s) for s in (113, 114, 115, 116))
+    bm = BLOCK_MASKS[0]
+    dq, dk, dv, _ = bwd(q, k, v, do, 0.8, True, None, bm)
+    h = 1e-6
+    worst = 0.0
+    for which, grad in ((0, dq), (1, dk), (2, dv)):
+        for idx in ((0, 0), (17, 2), (130, 1), (200, 0), (299, 2), (256, 1)):
+            args = [q.copy(), k.copy(), v.copy()]
+            args[which][idx] += h
+            lp = float(np.sum(do * A.forward_head(*args, 0.8, True, None, bm)[0]))
+            args[which][idx] -= 2 * h
+            lm = float(np.sum(do * A.forward_head(*args, 0.8, True, None, bm)[0]))
+            worst = max(worst, abs((lp - lm) / (2 * h) - grad[idx]))
+    return worst
+
+
 # ---------------------------------------------------------------------------
 # The pins themselves
 # ---------------------------------------------------------------------------
@@ -623,4 +672,36 @@ def test_window_mutants_are_caught(kind):
     if kind == "left_off_by_one":
         frac = window_skipped_block_fraction(32768, (4095, 0), 128, hidden=hidden)
         assert not (0.87 <= frac < 0.88) or _caught(pin_window_zero_width, fwd)
+
+
+def test_blocksparse_rows_equal_attention_over_their_blocks():
+    assert pin_blocksparse_rowwise() < 1e-12
+
+
+def test_blocksparse_special_cases():
+    n = 300
+    q, k, v = _rand((n, 4), 120), _rand((n, 4), 121), _rand((n, 4), 122)
+    full = A.forward_head(q, k, v, 0.5, False)
+    causal = A.forward_head(q, k, v, 0.5, True)
+    ones = np.ones((3, 3), dtype=np.uint8)
+    for a, b in zip(A.forward_head(q, k, v, 0.5, False, None, ones), full):
+        assert np.array_equal(a, b)
+    # block-lower-triangular mask on top of the causal mask hides nothing more
+    tril = np.tril(ones)
+    for a, b in zip(A.forward_head(q, k, v, 0.5, True, None, tril), causal):
+        assert np.array_equal(a, b)
+
+
+def test_blocksparse_backward_finite_differences():
+    assert pin_blocksparse_finite_differences() < 1e-7
+
+
+def test_blocksparse_mutants_are_caught():
+    def transposed_mask(q, k, v, scale, causal, window=None, block_mask=None):
+        return A.forward_head(q, k, v, scale, causal, window, None if block_mask is None else block_mask.T)
+    assert _caught(pin_blocksparse_rowwise, transposed_mask)
+
+    def dense(q, k, v, scale, causal, window=None, block_mask=None):
+        return A.forward_head(q, k, v, scale, causal, window, None)
+    assert _caught(pin_blocksparse_rowwise, dense)
 
