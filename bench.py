@@ -298,6 +298,35 @@ def run_ours(args, world, rank, local):
                 "traffic": read_profile_traffic(dom["key"]),
                 "flops_per_launch": dom["flops"], "ms_per_launch": dom["ms"]}
 
+    # ---- the 8-bit forward on the same workload (e4m3 codes, per-tensor scales) ----
+    fp8 = None
+    if hasattr(torch, "float8_e4m3fn"):
+        codes, scales = [], []
+        for t in (q, k, v):
+            s_t = float(t.float().abs().max()) / 448.0 or 1.0
+            codes.append((t.float() / s_t).to(torch.float8_e4m3fn))
+            scales.append(s_t)
+        o8 = torch.empty_like(o)
+        for _ in range(3):
+            fa.fwd_fp8(*codes, *scales, causal=causal, scale=scale, out=o8, lse=lse)
+        n8 = max(3, min(args.steps, 10))
+        e8a, e8b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier()
+        torch.cuda.synchronize()
+        e8a.record(stream)
+        for _ in range(n8):
+            fa.fwd_fp8(*codes, *scales, causal=causal, scale=scale, out=o8, lse=lse)
+        e8b.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        ms8 = slowest(e8a.elapsed_time(e8b)) / n8
+        tf8 = f / (ms8 * 1e-3) / 1e12
+        fp8 = {"tflops": tf8, "ms": ms8, "launches": n8, "peak": 2 * peak_burst,
+               "frac_of_peak": tf8 / (2 * peak_burst),
+               "peak_source": "bf16 burst x 2 (the nominal e4m3 / bf16 dense ratio)",
+               "inputs": "Q, K, V of the same workload as e4m3 codes with per-tensor scales"}
+        del codes, o8
+
     # ---- end to end through the public API with host buffers ----
     # Every step copies its four inputs from pinned host memory and its five
     # outputs back.  Two device buffer sets and two copy streams pipeline the
@@ -378,6 +407,7 @@ def run_ours(args, world, rank, local):
         "frac_of_peak": value / world / peak_burst,
         "peak_tflops": {"burst": peak_burst, "sustained": peak_sustained, "source": peak_src},
         "roofline": roofline,
+        "fwd_fp8": fp8,
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "steps": e_steps, "ms_per_step": e2e_ms / e_steps,
                 "how": "pinned host -> device inputs and device -> pinned host outputs every step, "
@@ -401,7 +431,8 @@ PROFILE_WORKLOAD = dict(B=1, H=64, N=4096, d=128)
 
 def run_profile_case(args):
     """Small case for ncu section captures: 2 x (forward, backward) on B1 H64 N4096 d128
-    (each tensor 64 MiB, so the five of them exceed the L2; < 1 GB on the device)."""
+    (each tensor 64 MiB, so the five of them exceed the L2; < 1 GB on the device), then
+    2 x the 8-bit forward on the same Q, K, V."""
     import torch
 
     import exact_io_aware_51_b200 as fa
@@ -412,6 +443,9 @@ def run_profile_case(args):
         for _ in range(2):
             o, lse = fa.fwd(q, k, v, causal=causal)
             fa.bwd(q, k, v, o, do, lse, causal=causal)
+    q8, k8, v8 = (t.to(torch.float8_e4m3fn) for t in (q, k, v))
+    for _ in range(2):
+        fa.fwd_fp8(q8, k8, v8, 1.0, 1.0, 1.0)
     torch.cuda.synchronize()
     rc, detail = fa.last_device_status()
     if rc != 0:

@@ -149,6 +149,11 @@ struct BwdBars {
   uint64_t stage_sync;  // the dQ drain warpgroup's internal barrier
   uint32_t tmem_base;
   int abort;
+  // block-sparse: first query row of tile i, in slot i % 4 (written by the
+  // loader before it arms q_full for the tile; read by the compute warps after
+  // their q_full wait)
+  int info_q0[4];
+  int sparse_nq;  // block-sparse: kept (query head, query tile) pairs of this key tile
 };
 static_assert(sizeof(BwdBars) <= 256, "barrier block");
 static_assert(BwdCfg::kOffDQS % 1024 == 0 && BwdCfg::kSmemBytes <= 232448, "shared memory layout");
@@ -180,6 +185,7 @@ __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wa
 // P^T / dS^T tile written by the two compute warpgroups.
 __device__ __forceinline__ uint32_t ts_col(int kk) { return (kk < 4) ? kk * 8 : 64 + (kk - 4) * 8; }
 
+template <bool kSparse>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
@@ -210,10 +216,30 @@ __global__ void __launch_bounds__(kThreads, 1)
   // this CTA's dK and dV, so the CTA walks (query head, query tile) pairs.
   const int G = a.H / a.Hkv;
   const int nq_head = max(0, min(nq_total, i_end) - i0);  // query tiles per query head
-  const int nq = G * nq_head;                 // iterations of this CTA
+  int nq = G * nq_head;                       // iterations of this CTA
   // Iteration i works on query tile i0 + i % nq_head of query head hk G + i / nq_head;
   // the loops advance (qt, hq) by counters (a division per tile measurably slowed them).
+  // Block-sparse: only the (query head, query tile) pairs the mask keeps for this key
+  // tile, in the same order; the loader walks them and posts each tile's (q0, head).
   const int qt_end = i0 + nq_head;
+  auto kept = [&](int hq, int qt) -> bool {
+    return a.block_mask[(static_cast<size_t>(a.mask_heads == 1 ? 0 : hq) * a.nb + qt) * a.nb + jt] != 0;
+  };
+  if constexpr (kSparse) {
+    // (a static __shared__ variable here would push the 1024-aligned dynamic
+    // region past the shared-memory limit, so the count lives in the barrier block)
+    int& s_nq = bars->sparse_nq;
+    if (threadIdx.x == 0) s_nq = 0;
+    __syncthreads();
+    int cnt = 0;
+    for (int c = static_cast<int>(threadIdx.x); c < nq; c += kThreads)
+      cnt += kept(hk * G + c / nq_head, i0 + c % nq_head) ? 1 : 0;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+    if (lane == 0 && cnt) atomicAdd(&s_nq, cnt);
+    __syncthreads();
+    nq = s_nq;
+  }
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->kv_full, 1);
@@ -258,10 +284,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int i = 0; i < nq; ++i) {
         const int st = i % kStages;
         const uint32_t par = i & 1;
-        const int q0 = qt * kBMq + 64 * g;  // first query column of this WG
+        int q0 = qt * kBMq + 64 * g;  // first query column of this WG
         qt = (qt + 1 == qt_end) ? i0 : qt + 1;
         ok = warp_all(wait_bar(&bars->q_full[st], (i / kStages) & 1, w, 20));
         if (!ok) break;
+        if constexpr (kSparse) q0 = *reinterpret_cast<volatile int*>(&bars->info_q0[i & 3]) + 64 * g;
         ok = warp_all(wait_bar(&bars->s_full, par, w, 21));
         if (!ok) break;
         tc_fence_after();
@@ -408,6 +435,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         return r;
       };
       int qt = i0, hq = hk * G;
+      if constexpr (kSparse) {
+        while (hq < hk * G + G && !kept(hq, qt)) {
+          if (++qt == qt_end) {
+            qt = i0;
+            ++hq;
+          }
+        }
+      }
       for (int i = 0; ok && i < nq; ++i) {
         if (!(ok = warp_all(wait_bar(&bars->dq_full, i & 1, w, 30)))) break;
         tc_fence_after();
@@ -433,10 +468,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             bulk_commit();
           }
         }
-        if (++qt == qt_end) {
-          qt = i0;
-          ++hq;
-        }
+        do {
+          if (++qt == qt_end) {
+            qt = i0;
+            ++hq;
+          }
+        } while (kSparse && hq < hk * G + G && !kept(hq, qt));
       }
       if (issuer) bulk_wait_all();
     }
@@ -455,16 +492,27 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_4d(smem + C::kOffV + c * C::kSub, &tmV, &bars->kv_full, c * 64, key0, hk, b);
         }
         int qt = i0, hq = hk * G;
+        if constexpr (kSparse) {
+          while (hq < hk * G + G && !kept(hq, qt)) {
+            if (++qt == qt_end) {
+              qt = i0;
+              ++hq;
+            }
+          }
+        }
         for (int i = 0; i < nq; ++i) {
           const int st = i % kStages;
           const int n = i / kStages;
           const int q0 = qt * kBMq;
           const int hq_i = hq;
-          if (++qt == qt_end) {
-            qt = i0;
-            ++hq;
-          }
+          do {
+            if (++qt == qt_end) {
+              qt = i0;
+              ++hq;
+            }
+          } while (kSparse && hq < hk * G + G && !kept(hq, qt));
           if (i >= kStages && !wait_bar(&bars->q_empty[st], (n - 1) & 1, w, 10)) break;
+          if constexpr (kSparse) bars->info_q0[i & 3] = q0;
           const size_t bh = static_cast<size_t>(b) * a.H + hq_i;
           mbar_arrive_expect_tx(&bars->q_full[st], 2 * C::kTile + 1024);
           for (int c = 0; c < D / 64; ++c) {
@@ -578,11 +626,14 @@ cudaError_t launch_bwd_main(const CUtensorMap& tq, const CUtensorMap& tk, const 
                             const CUtensorMap& tdo, const CUtensorMap& tdq, const BwdArgs& a, const DevCtl& c,
                             cudaStream_t s) {
   constexpr int smem = BwdCfg::kSmemBytes;
-  cudaError_t e = cudaFuncSetAttribute(bwd_main_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e != cudaSuccess) return e;
   const dim3 grid((a.N + kBN - 1) / kBN, a.Hkv, a.B);
-  bwd_main_kernel<<<grid, kThreads, smem, s>>>(tq, tk, tv, tdo, tdq, a, c);
-  return cudaGetLastError();
+  auto run = [&](auto kernel) -> cudaError_t {
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    kernel<<<grid, kThreads, smem, s>>>(tq, tk, tv, tdo, tdq, a, c);
+    return cudaGetLastError();
+  };
+  return a.block_mask ? run(bwd_main_kernel<true>) : run(bwd_main_kernel<false>);
 }
 
 cudaError_t launch_bwd_dq(const BwdArgs& a, cudaStream_t s) {

@@ -63,7 +63,9 @@ struct FwdCfg {
   static constexpr int kOffK = 2 * kTileBytes;
   static constexpr int kOffV = kOffK + kStages * kTileBytes;
   static constexpr int kOffBar = kOffV + kStages * kTileBytes;
+  static constexpr int kOffList = kOffBar + 512;           // block-sparse: the CTA's key-tile list
   static constexpr int kSmemBytes = kOffBar + 512 + 1024;  // barriers + base alignment slack
+  static constexpr int kSmemBytesSparse = kOffList + 4 * kMaxSparseTiles + 1024;
   // TMEM columns: S_0 | S_1 | O_0 | O_1
   __device__ static constexpr uint32_t colS(int t) { return static_cast<uint32_t>(t) * 128u; }
   __device__ static constexpr uint32_t colO(int t) { return 256u + static_cast<uint32_t>(t) * D; }
@@ -91,7 +93,7 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, unsig
 
 __device__ __forceinline__ bool warp_all(bool ok) { return __all_sync(0xffffffffu, ok); }
 
-template <int D>
+template <int D, bool kSparse>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const FwdArgs a, const DevCtl ctl) {
@@ -124,7 +126,56 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
   const int kbase = klo[0];
-  const int nk = (nkt[1] > 0) ? max(klo[0] + nkt[0], klo[1] + nkt[1]) - kbase : nkt[0];
+  int nk = (nkt[1] > 0) ? max(klo[0] + nkt[0], klo[1] + nkt[1]) - kbase : nkt[0];
+
+  // Block-sparse: the key tiles of the window range that the mask keeps for at
+  // least one of the two query tiles, in ascending order, as (tile << 2 | bits)
+  // with bit t set when query tile t uses the tile.  All roles read this list;
+  // nkt[t] becomes query tile t's count and nk the stream length.
+  const uint32_t* klist = reinterpret_cast<const uint32_t*>(smem + C::kOffList);
+  if constexpr (kSparse) {
+    uint32_t* list = reinterpret_cast<uint32_t*>(smem + C::kOffList);
+    __shared__ int s_wcnt[kThreads / 32];
+    __shared__ int s_cnt[3];
+    const uint8_t* mrow0 = a.block_mask + (static_cast<size_t>(a.mask_heads == 1 ? 0 : h) * a.nb + q0[0] / kBM) * a.nb;
+    const uint8_t* mrow1 = mrow0 + a.nb;
+    if (threadIdx.x < 3) s_cnt[threadIdx.x] = 0;
+    __syncthreads();
+    for (int base = 0; base < nk; base += kThreads) {
+      const int c = base + static_cast<int>(threadIdx.x);
+      const int kt = kbase + c;
+      uint32_t f = 0;
+      if (c < nk) {
+        if (kt >= klo[0] && kt < klo[0] + nkt[0] && mrow0[kt]) f |= 1u;
+        if (kt >= klo[1] && kt < klo[1] + nkt[1] && mrow1[kt]) f |= 2u;
+      }
+      const unsigned bal = __ballot_sync(0xffffffffu, f != 0);
+      if (lane == 0) s_wcnt[warp] = __popc(bal);
+      __syncthreads();
+      int off = s_cnt[2];
+      for (int w2 = 0; w2 < warp; ++w2) off += s_wcnt[w2];
+      if (f) {
+        list[off + __popc(bal & ((1u << lane) - 1u))] = (static_cast<uint32_t>(kt) << 2) | f;
+        if (f & 1u) atomicAdd(&s_cnt[0], 1);
+        if (f & 2u) atomicAdd(&s_cnt[1], 1);
+      }
+      __syncthreads();
+      if (threadIdx.x == 0) {
+        int tot = 0;
+        for (int w2 = 0; w2 < kThreads / 32; ++w2) tot += s_wcnt[w2];
+        s_cnt[2] += tot;
+      }
+      __syncthreads();
+    }
+    nkt[0] = s_cnt[0];
+    nkt[1] = s_cnt[1];
+    nk = s_cnt[2];
+  }
+  // key tile of stream position j, and whether query tile t uses it (dense: the window ranges)
+  auto stream_tile = [&](int j) -> int { return kSparse ? static_cast<int>(klist[j] >> 2) : kbase + j; };
+  auto uses = [&](int t, int j) -> bool {
+    return kSparse ? ((klist[j] >> t) & 1u) != 0 : (kbase + j >= klo[t] && kbase + j < klo[t] + nkt[t]);
+  };
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
@@ -166,7 +217,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       float m = -INFINITY;
       float l = 0.f;
       bool ok = true;
+      int e = -1;  // stream position of this tile's j-th key tile
       for (int j = 0; j < nkt[t]; ++j) {
+        if constexpr (kSparse) {
+          do {
+            ++e;
+          } while (!uses(t, e));
+        } else {
+          e = klo[t] - kbase + j;
+        }
         ok = warp_all(wait_bar(&bars->s_full[t], j & 1, w, 8));
         if (!ok) break;
         tc_fence_after();
@@ -177,7 +236,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int c = 0; c < kBN / 32; ++c) reg_fence32(sr + c * 32);
 
-        const int k0 = (klo[t] + j) * kBN;
+        const int k0 = stream_tile(e) * kBN;
         // whole tile visible to every row of the query tile: no mask
         const bool need_mask = (k0 + kBN > a.N) || (k0 + kBN - 1 > q0[t] + a.wr) || (k0 < q0[t] + kBM - 1 - a.wl);
         if (need_mask) {
@@ -251,6 +310,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(&bars->p_full[t]);
       }
       // ---- epilogue ----
+      if (ok && nkt[t] == 0 && qrow < a.N) {
+        // block-sparse: no key is visible to this row: O = 0, LSE = -inf
+        __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.O) + ((static_cast<size_t>(b) * a.N + qrow) * a.H + h) * D;
+#pragma unroll
+        for (int c = 0; c < D; c += 8) st_global_v4(orow + c, 0u, 0u, 0u, 0u);
+        a.LSE[(static_cast<size_t>(b) * a.H + h) * a.N + qrow] = -INFINITY;
+      }
       if (ok && nkt[t] > 0) {
         ok = warp_all(wait_bar(&bars->o_done[t], (nkt[t] - 1) & 1, w, 9));
         if (ok) {
@@ -306,12 +372,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive_expect_tx(&bars->k_full[s], C::kTileBytes + extra);
           for (int c = 0; c < C::kSub; ++c)
             tma_load_4d(smem + C::kOffK + s * C::kTileBytes + c * C::kSubBytes, &tmK, &bars->k_full[s], c * 64,
-                        (kbase + j) * kBN, hk, b);
+                        stream_tile(j) * kBN, hk, b);
           if (j >= C::kStages && !wait_bar(&bars->v_empty[s], (n - 1) & 1, w, 2)) break;
           mbar_arrive_expect_tx(&bars->v_full[s], C::kTileBytes);
           for (int c = 0; c < C::kSub; ++c)
             tma_load_4d(smem + C::kOffV + s * C::kTileBytes + c * C::kSubBytes, &tmV, &bars->v_full[s], c * 64,
-                        (kbase + j) * kBN, hk, b);
+                        stream_tile(j) * kBN, hk, b);
         }
       }
     } else if (warp == 9) {
@@ -342,20 +408,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           umma_commit(&bars->o_done[t]);
         };
-        // Stream tile j is key tile kbase + j; for query tile t it is local
-        // tile j - (klo[t] - kbase), active when that lies in [0, nkt[t]).
-        auto local = [&](int t, int j) { return j - (klo[t] - kbase); };
-        auto active = [&](int t, int j) { return local(t, j) >= 0 && local(t, j) < nkt[t]; };
+        // jl[t]: how many of query tile t's key tiles have had their P V issued
+        int jl[2] = {0, 0};
         // Issue order: S_0(0) S_1(0) | PV_0(j) S_0(j+1) PV_1(j) S_1(j+1) | ...
         // S_t(j+1) overwrites the columns PV_t(j) reads P_t(j) from; the tensor
         // pipe executes one thread's MMAs in issue order, so PV_t(j) has read
         // P_t(j) before S_t(j+1) writes there.  A query tile whose first key
         // tile is a later stream tile gets its first S in the iteration before.
-        bool ok = wait_bar(&bars->q_full, 0, w, 3) && wait_bar(&bars->k_full[0], 0, w, 4);
+        bool ok = nk > 0 && wait_bar(&bars->q_full, 0, w, 3) && wait_bar(&bars->k_full[0], 0, w, 4);
         if (ok) {
           tc_fence_after();
           for (int t = 0; t < 2; ++t)
-            if (active(t, 0)) issue_s(t, 0);
+            if (uses(t, 0)) issue_s(t, 0);
           umma_commit(&bars->k_empty[0]);
         }
         for (int j = 0; ok && j < nk; ++j) {
@@ -364,13 +428,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!(ok = wait_bar(&bars->v_full[s], (j / C::kStages) & 1, w, 6))) break;
           bool next_k = false;
           for (int t = 0; t < 2; ++t) {
-            if (active(t, j)) {
-              const int jl = local(t, j);
-              if (!(ok = wait_bar(&bars->p_full[t], jl & 1, w, 7))) break;
+            if (uses(t, j)) {
+              if (!(ok = wait_bar(&bars->p_full[t], jl[t] & 1, w, 7))) break;
               tc_fence_after();
-              issue_pv(t, s, jl > 0);
+              issue_pv(t, s, jl[t] > 0);
+              ++jl[t];
             }
-            if (j + 1 < nk && active(t, j + 1)) {
+            if (j + 1 < nk && uses(t, j + 1)) {
               if (!next_k) {
                 if (!(ok = wait_bar(&bars->k_full[sn], ((j + 1) / C::kStages) & 1, w, 5))) break;
                 tc_fence_after();
@@ -404,18 +468,18 @@ cudaError_t launch_fwd_bf16(const CUtensorMap& tq, const CUtensorMap& tk, const 
                             const DevCtl& c, cudaStream_t s) {
   const int nqb = (a.N + 2 * kBM - 1) / (2 * kBM);
   const dim3 grid(nqb, a.H, a.B);
-  if (a.d == 128) {
-    constexpr int smem = FwdCfg<128>::kSmemBytes;
-    cudaError_t e = cudaFuncSetAttribute(fwd_bf16_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  auto run = [&](auto kernel, int smem) -> cudaError_t {
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    fwd_bf16_kernel<128><<<grid, kThreads, smem, s>>>(tq, tk, tv, a, c);
-  } else {
-    constexpr int smem = FwdCfg<64>::kSmemBytes;
-    cudaError_t e = cudaFuncSetAttribute(fwd_bf16_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    fwd_bf16_kernel<64><<<grid, kThreads, smem, s>>>(tq, tk, tv, a, c);
-  }
-  return cudaGetLastError();
+    kernel<<<grid, kThreads, smem, s>>>(tq, tk, tv, a, c);
+    return cudaGetLastError();
+  };
+  const bool sparse = a.block_mask != nullptr;
+  if (a.d == 128)
+    return sparse ? run(fwd_bf16_kernel<128, true>, FwdCfg<128>::kSmemBytesSparse)
+                  : run(fwd_bf16_kernel<128, false>, FwdCfg<128>::kSmemBytes);
+  return sparse ? run(fwd_bf16_kernel<64, true>, FwdCfg<64>::kSmemBytesSparse)
+                : run(fwd_bf16_kernel<64, false>, FwdCfg<64>::kSmemBytes);
 }
 
 }  // namespace fa

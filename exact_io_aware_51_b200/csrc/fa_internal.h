@@ -31,7 +31,15 @@ struct FwdArgs {
   int wl, wr;        // window (see above)
   void* O;           // [B, N, H, d]
   float* LSE;        // [B, H, N], natural log
+  // Block-sparse mask (nullptr: none): [mask_heads][nb][nb] bytes, nb = ceil(N / 128);
+  // query tile i sees key tile j of query head h when mask[(mh * nb + i) * nb + j] != 0
+  // with mh = (mask_heads == 1 ? 0 : h).
+  const uint8_t* block_mask;
+  int mask_heads, nb;
 };
+
+// Largest key-tile count (ceil(N / 128)) the block-sparse kernels accept.
+constexpr int kMaxSparseTiles = 4096;
 
 struct BwdArgs {
   int B, H, N, d, Npad;
@@ -49,6 +57,8 @@ struct BwdArgs {
   float* dQacc;      // [B, N, H, d] fp32 workspace
   float* Dvec;       // [B, H, Npad] rowsum(dO * O)
   float* LSE2;       // [B, H, Npad] LSE * log2(e)
+  const uint8_t* block_mask;  // as in FwdArgs (nullptr: none)
+  int mask_heads, nb;
 };
 
 // TMA descriptor for a [B, N, H, d] bf16 tensor with a box of `rows` sequence
@@ -74,6 +84,12 @@ cudaError_t launch_bwd_main(const CUtensorMap& tq, const CUtensorMap& tk, const 
                             const CUtensorMap& tdo, const CUtensorMap& tdq, const BwdArgs& a, const DevCtl& c,
                             cudaStream_t s);
 cudaError_t launch_bwd_dq(const BwdArgs& a, cudaStream_t s);
+
+// Chunked-sequence (ring) helpers: merge of partial results, fp32 accumulation, cast.
+cudaError_t launch_merge(float* o_acc, float* lse_acc, const void* o_part, const float* lse_part, void* o_out, int B,
+                         int H, int N, int d, int init, cudaStream_t s);
+cudaError_t launch_accumulate(float* acc, const void* part, long long n, int init, cudaStream_t s);
+cudaError_t launch_cast(void* out, const float* in, long long n, cudaStream_t s);
 
 // Test-only single-tile MMA probe (see fa_debug_umma in the public header).
 cudaError_t launch_umma_probe(const void* A, const void* B, float* D, int N, int K, int a_mn_major,

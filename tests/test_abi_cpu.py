@@ -188,3 +188,20 @@ def test_fp8_forward_validation(L):
     assert f(16, 16, 16, 16, 16, 1, 4, 2, 128, 128, 0.1, *ok, -3, -1, None) == -1
     assert f(8, 16, 16, 16, 16, 1, 4, 2, 128, 128, 0.1, *ok, 64, 0, None) == -3
     assert f(None, None, None, None, None, 0, 4, 2, 128, 128, 0.1, *ok, -1, -1, None) == 0
+
+
+def test_blocksparse_validation(L):
+    """fa_fwd_blocksparse / fa_bwd_blocksparse argument checks (no device work)."""
+    f = L.fa_fwd_blocksparse
+    # null mask, wrong mask_heads, fp32, too many key blocks
+    assert f(16, 16, 16, 16, 16, 1, 4, 4, 256, 128, 0.1, -1, -1, None, 1, 0, None) == -1
+    assert f(16, 16, 16, 16, 16, 1, 4, 4, 256, 128, 0.1, -1, -1, 16, 2, 0, None) == -1
+    assert f(16, 16, 16, 16, 16, 1, 4, 4, 256, 128, 0.1, -1, -1, 16, 1, 1, None) == -2
+    assert f(16, 16, 16, 16, 16, 1, 4, 4, 4096 * 128 + 1, 128, 0.1, -1, -1, 16, 1, 0, None) == -8
+    # valid arguments reach the alignment check
+    assert f(8, 16, 16, 16, 16, 1, 4, 4, 256, 128, 0.1, -1, -1, 16, 4, 0, None) == -3
+    b = L.fa_bwd_blocksparse
+    args = [16] * 9
+    ws = L.fa_bwd_workspace_size(1, 4, 256, 128, 0)
+    assert b(*args, 1, 4, 4, 256, 128, 0.1, -1, -1, None, 1, 0, 256, ws, None) == -1
+    assert b(*args, 1, 4, 4, 256, 128, 0.1, -1, -1, 16, 3, 0, 256, ws, None) == -1
