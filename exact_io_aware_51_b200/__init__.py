@@ -20,6 +20,7 @@ import torch
 
 __all__ = [
     "FAError", "FA_BF16", "FA_FP32", "lib", "lib_path", "fwd", "fwd_fp8", "bwd", "bwd_workspace_size",
+    "merge_partial", "accumulate", "cast_bf16",
     "last_device_status", "set_wait_limit_ms", "debug_inject", "debug_umma", "debug_umma_f8", "status_string",
     "set_kernel_events",
     "attention", "EXPORTED",
@@ -34,7 +35,9 @@ _LIB = None
 EXPORTED = ("fa_fwd", "fa_bwd_workspace_size", "fa_bwd", "fa_status_string", "fa_last_cuda_error",
             "fa_last_device_status", "fa_set_wait_limit_ms", "fa_debug_inject", "fa_debug_umma",
             "fa_version", "fa_set_kernel_events", "fa_bwd_static_scratch", "fa_fwd_gqa", "fa_bwd_gqa",
-            "fa_fwd_window", "fa_bwd_window", "fa_debug_umma_f8", "fa_fwd_fp8")
+            "fa_fwd_window", "fa_bwd_window", "fa_debug_umma_f8", "fa_fwd_fp8",
+            "fa_fwd_blocksparse", "fa_bwd_blocksparse", "fa_merge_partial", "fa_accumulate_bf16",
+            "fa_cast_bf16")
 
 
 class FAError(RuntimeError):
@@ -74,6 +77,16 @@ def lib() -> ctypes.CDLL:
     L.fa_bwd_gqa.restype = i
     L.fa_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, f, f, f, i, i, vp]
     L.fa_fwd_fp8.restype = i
+    L.fa_fwd_blocksparse.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp, i, i, vp]
+    L.fa_fwd_blocksparse.restype = i
+    L.fa_bwd_blocksparse.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp, i, i, vp, sz, vp]
+    L.fa_bwd_blocksparse.restype = i
+    L.fa_merge_partial.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, vp]
+    L.fa_merge_partial.restype = i
+    L.fa_accumulate_bf16.argtypes = [vp, vp, ctypes.c_longlong, i, vp]
+    L.fa_accumulate_bf16.restype = i
+    L.fa_cast_bf16.argtypes = [vp, vp, ctypes.c_longlong, vp]
+    L.fa_cast_bf16.restype = i
     L.fa_fwd_window.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, i, vp]
     L.fa_fwd_window.restype = i
     L.fa_bwd_window.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, i, vp, sz, vp]
@@ -154,13 +167,30 @@ def _window_bounds(causal, window):
     return (-1 if left is None else int(left)), (-1 if right is None else int(right))
 
 
+def _mask_args(block_mask, q):
+    """(pointer, mask_heads) for a uint8 cuda block mask [nb, nb] or [H, nb, nb]."""
+    B, N, H, d = q.shape
+    nb = (N + 127) // 128
+    if block_mask.dtype not in (torch.uint8, torch.bool) or not block_mask.is_contiguous():
+        raise ValueError("block_mask must be a contiguous uint8 (or bool) tensor")
+    if block_mask.device != q.device:
+        raise ValueError("block_mask must live on the device of q")
+    if block_mask.shape == (nb, nb):
+        return block_mask.data_ptr(), 1
+    if block_mask.shape == (H, nb, nb):
+        return block_mask.data_ptr(), H
+    raise ValueError(f"block_mask must be [{nb}, {nb}] or [{H}, {nb}, {nb}] (128 x 128 blocks)")
+
+
 def fwd(q, k, v, causal: bool = False, scale: float | None = None, out=None, lse=None, stream=None,
-        window=None):
+        window=None, block_mask=None):
     """Forward pass: returns (o [B, N, H, d], lse [B, H, N] fp32).
 
     k and v may have fewer heads than q (grouped-query attention, fa_fwd_gqa).
     ``window`` = (left, right) restricts query i to keys i - left .. i + right
-    (None on a side: open), fa_fwd_window.
+    (None on a side: open), fa_fwd_window.  ``block_mask`` (uint8 [nb, nb] or
+    [H, nb, nb] over 128 x 128 blocks) selects the blocks each query block sees,
+    fa_fwd_blocksparse.
     """
     Hkv = _check_inputs(q, k, v)
     B, N, H, d = q.shape
@@ -168,7 +198,12 @@ def fwd(q, k, v, causal: bool = False, scale: float | None = None, out=None, lse
     l = torch.empty((B, H, N), dtype=torch.float32, device=q.device) if lse is None else lse
     tail = (_scale(scale, d), int(bool(causal)), _dtype_code(q), _stream_handle(stream, q.device))
     ptrs = (q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), l.data_ptr())
-    if window is not None:
+    if block_mask is not None:
+        wl, wr = _window_bounds(causal, (None, None) if window is None else window)
+        mp, mh = _mask_args(block_mask, q)
+        rc, name = lib().fa_fwd_blocksparse(*ptrs, B, H, Hkv, N, d, tail[0], wl, wr, mp, mh, *tail[2:]), \
+            "fa_fwd_blocksparse"
+    elif window is not None:
         wl, wr = _window_bounds(causal, window)
         rc, name = lib().fa_fwd_window(*ptrs, B, H, Hkv, N, d, tail[0], wl, wr, *tail[2:]), "fa_fwd_window"
     elif Hkv == H:
@@ -200,12 +235,50 @@ def fwd_fp8(q, k, v, scale_q: float, scale_k: float, scale_v: float, causal: boo
     return o, l
 
 
+def merge_partial(o_acc, lse_acc, o_part, lse_part, init: bool = False, o_out=None, stream=None):
+    """Fold one key chunk's partial result (o_part bf16, lse_part) into (o_acc fp32, lse_acc), in place."""
+    B, N, H, d = o_part.shape
+    for t, dt in ((o_acc, torch.float32), (lse_acc, torch.float32), (o_part, torch.bfloat16), (lse_part, torch.float32)):
+        if t.dtype != dt or not t.is_contiguous() or not t.is_cuda:
+            raise ValueError("merge_partial: contiguous cuda tensors (o_acc fp32, o_part bf16, LSEs fp32)")
+    if o_acc.shape != o_part.shape or lse_acc.shape != (B, H, N) or lse_part.shape != (B, H, N):
+        raise ValueError("merge_partial: shape mismatch")
+    rc = lib().fa_merge_partial(o_acc.data_ptr(), lse_acc.data_ptr(), o_part.data_ptr(), lse_part.data_ptr(),
+                                None if o_out is None else o_out.data_ptr(), B, H, N, d, int(bool(init)),
+                                _stream_handle(stream, o_acc.device))
+    if rc != 0:
+        raise FAError(rc, "fa_merge_partial")
+
+
+def accumulate(acc, part, init: bool = False, stream=None):
+    """acc (fp32) += part (bf16), or acc = part with init; same shapes, contiguous cuda tensors."""
+    if acc.dtype != torch.float32 or part.dtype != torch.bfloat16 or acc.shape != part.shape:
+        raise ValueError("accumulate: fp32 accumulator and bf16 part of one shape")
+    if not (acc.is_cuda and part.is_cuda and acc.is_contiguous() and part.is_contiguous()):
+        raise ValueError("accumulate: contiguous cuda tensors")
+    rc = lib().fa_accumulate_bf16(acc.data_ptr(), part.data_ptr(), acc.numel(), int(bool(init)),
+                                  _stream_handle(stream, acc.device))
+    if rc != 0:
+        raise FAError(rc, "fa_accumulate_bf16")
+
+
+def cast_bf16(x, out=None, stream=None):
+    """bf16 copy of a contiguous fp32 cuda tensor (round to nearest even)."""
+    if x.dtype != torch.float32 or not x.is_cuda or not x.is_contiguous():
+        raise ValueError("cast_bf16: contiguous fp32 cuda tensor")
+    out = torch.empty(x.shape, dtype=torch.bfloat16, device=x.device) if out is None else out
+    rc = lib().fa_cast_bf16(out.data_ptr(), x.data_ptr(), x.numel(), _stream_handle(stream, x.device))
+    if rc != 0:
+        raise FAError(rc, "fa_cast_bf16")
+    return out
+
+
 def bwd_workspace_size(B: int, H: int, N: int, d: int, dtype: int = FA_BF16) -> int:
     return int(lib().fa_bwd_workspace_size(B, H, N, d, dtype))
 
 
 def bwd(q, k, v, o, do, lse, causal: bool = False, scale: float | None = None, workspace=None,
-        dq=None, dk=None, dv=None, stream=None, window=None):
+        dq=None, dk=None, dv=None, stream=None, window=None, block_mask=None):
     """Backward pass by recomputation: returns (dq, dk, dv), shaped like (q, k, v).
 
     With fewer K/V heads than query heads (fa_bwd_gqa), dk and dv are summed
@@ -226,7 +299,12 @@ def bwd(q, k, v, o, do, lse, causal: bool = False, scale: float | None = None, w
             dq.data_ptr(), dk.data_ptr(), dv.data_ptr())
     tail = (_scale(scale, d), int(bool(causal)), _dtype_code(q), workspace.data_ptr(), workspace.numel(),
             _stream_handle(stream, q.device))
-    if window is not None:
+    if block_mask is not None:
+        wl, wr = _window_bounds(causal, (None, None) if window is None else window)
+        mp, mh = _mask_args(block_mask, q)
+        rc, name = lib().fa_bwd_blocksparse(*ptrs, B, H, Hkv, N, d, tail[0], wl, wr, mp, mh, *tail[2:]), \
+            "fa_bwd_blocksparse"
+    elif window is not None:
         wl, wr = _window_bounds(causal, window)
         rc, name = lib().fa_bwd_window(*ptrs, B, H, Hkv, N, d, tail[0], wl, wr, *tail[2:]), "fa_bwd_window"
     elif Hkv == H:
@@ -285,20 +363,21 @@ def debug_umma_f8(a: torch.Tensor, b: torch.Tensor, b_mn_major: int, a_tmem: int
 
 class _Attention(torch.autograd.Function):
     @staticmethod
-    def forward(ctx, q, k, v, causal, scale, window):
-        o, lse = fwd(q, k, v, causal=causal, scale=scale, window=window)
+    def forward(ctx, q, k, v, causal, scale, window, block_mask):
+        o, lse = fwd(q, k, v, causal=causal, scale=scale, window=window, block_mask=block_mask)
         ctx.save_for_backward(q, k, v, o, lse)
-        ctx.causal, ctx.scale, ctx.window = causal, scale, window
+        ctx.causal, ctx.scale, ctx.window, ctx.block_mask = causal, scale, window, block_mask
         return o
 
     @staticmethod
     def backward(ctx, do):
         q, k, v, o, lse = ctx.saved_tensors
-        dq, dk, dv = bwd(q, k, v, o, do.contiguous(), lse, causal=ctx.causal, scale=ctx.scale, window=ctx.window)
-        return dq, dk, dv, None, None, None
+        dq, dk, dv = bwd(q, k, v, o, do.contiguous(), lse, causal=ctx.causal, scale=ctx.scale, window=ctx.window,
+                         block_mask=ctx.block_mask)
+        return dq, dk, dv, None, None, None, None
 
 
-def attention(q, k, v, causal: bool = False, scale: float | None = None, window=None):
+def attention(q, k, v, causal: bool = False, scale: float | None = None, window=None, block_mask=None):
     """Differentiable attention: q [B, N, H, d], k and v [B, N, Hkv, d] (Hkv divides H);
-    optional sliding ``window`` = (left, right)."""
-    return _Attention.apply(q, k, v, causal, scale, window)
+    optional sliding ``window`` = (left, right) and 128 x 128 ``block_mask``."""
+    return _Attention.apply(q, k, v, causal, scale, window, block_mask)

@@ -275,12 +275,27 @@ int fa_last_device_status(void* stream, int* detail) {
   return v ? FA_ERR_DEVICE_TIMEOUT : FA_OK;
 }
 
-int fa_fwd_window(const void* Q, const void* K, const void* V, void* O, float* LSE, int B, int H, int Hkv, int N,
-                  int d, float scale, int window_left, int window_right, int dtype, void* stream) {
+}  // extern "C"
+
+namespace {
+// Block-sparse mask checks: mask_heads is 1 or H and the key-tile count fits the
+// kernels' per-CTA list.  A null mask means no mask.
+int check_mask(const uint8_t* mask, int mask_heads, int H, int N, int dtype) {
+  if (!mask) return FA_OK;
+  if (dtype != FA_BF16) return FA_ERR_UNSUPPORTED;
+  if (mask_heads != 1 && mask_heads != H) return FA_ERR_INVALID_ARG;
+  if ((N + 127) / 128 > kMaxSparseTiles) return FA_ERR_TOO_LARGE;
+  return FA_OK;
+}
+
+int fwd_common(const void* Q, const void* K, const void* V, void* O, float* LSE, int B, int H, int Hkv, int N, int d,
+               float scale, int window_left, int window_right, const uint8_t* mask, int mask_heads, int dtype,
+               void* stream) {
   int rc = check_shape(B, H, N, d, dtype);
   if (rc) return rc;
   if ((rc = check_kv_heads(H, Hkv))) return rc;
   if ((rc = check_window(window_left, window_right))) return rc;
+  if ((rc = check_mask(mask, mask_heads, H, N, dtype))) return rc;
   if ((rc = check_scale(scale))) return rc;
   if (static_cast<long long>(B) * H * N == 0) return FA_OK;
   if (!Q || !K || !V || !O || !LSE) return FA_ERR_INVALID_ARG;
@@ -299,6 +314,9 @@ int fa_fwd_window(const void* Q, const void* K, const void* V, void* O, float* L
   set_window(window_left, window_right, &a.wl, &a.wr, &a.causal);
   a.O = O;
   a.LSE = LSE;
+  a.block_mask = mask;
+  a.mask_heads = mask_heads;
+  a.nb = (N + 127) / 128;
   cudaError_t e;
   if (dtype == FA_FP32) {
     e = launch_fwd_f32(static_cast<const float*>(Q), static_cast<const float*>(K), static_cast<const float*>(V), a, s);
@@ -315,6 +333,23 @@ int fa_fwd_window(const void* Q, const void* K, const void* V, void* O, float* L
   }
   if (e != cudaSuccess) return fail_cuda(e);
   return FA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int fa_fwd_window(const void* Q, const void* K, const void* V, void* O, float* LSE, int B, int H, int Hkv, int N,
+                  int d, float scale, int window_left, int window_right, int dtype, void* stream) {
+  return fwd_common(Q, K, V, O, LSE, B, H, Hkv, N, d, scale, window_left, window_right, nullptr, 0, dtype, stream);
+}
+
+int fa_fwd_blocksparse(const void* Q, const void* K, const void* V, void* O, float* LSE, int B, int H, int Hkv, int N,
+                       int d, float scale, int window_left, int window_right, const void* block_mask,
+                       int mask_heads, int dtype, void* stream) {
+  if (!block_mask && static_cast<long long>(B) * H * N > 0) return FA_ERR_INVALID_ARG;
+  return fwd_common(Q, K, V, O, LSE, B, H, Hkv, N, d, scale, window_left, window_right,
+                    static_cast<const uint8_t*>(block_mask), mask_heads, dtype, stream);
 }
 
 int fa_fwd_gqa(const void* Q, const void* K, const void* V, void* O, float* LSE, int B, int H, int Hkv, int N, int d,
@@ -355,6 +390,9 @@ int fa_fwd_fp8(const void* Q, const void* K, const void* V, void* O, float* LSE,
   set_window(window_left, window_right, &a.wl, &a.wr, &a.causal);
   a.O = O;
   a.LSE = LSE;
+  a.block_mask = nullptr;
+  a.mask_heads = 0;
+  a.nb = (N + 127) / 128;
   CUtensorMap tq, tk, tv;
   CUresult r;
   if ((r = make_tile_map_e4m3(&tq, Q, B, N, H, d, 128)) != CUDA_SUCCESS ||
@@ -377,13 +415,18 @@ size_t fa_bwd_workspace_size(int B, int H, int N, int d, int dtype) {
   return dq + 2 * rows;
 }
 
-int fa_bwd_window(const void* Q, const void* K, const void* V, const void* O, const void* dO, const float* LSE,
-                  void* dQ, void* dK, void* dV, int B, int H, int Hkv, int N, int d, float scale, int window_left,
-                  int window_right, int dtype, void* workspace, size_t workspace_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+int bwd_common(const void* Q, const void* K, const void* V, const void* O, const void* dO, const float* LSE,
+               void* dQ, void* dK, void* dV, int B, int H, int Hkv, int N, int d, float scale, int window_left,
+               int window_right, const uint8_t* mask, int mask_heads, int dtype, void* workspace,
+               size_t workspace_bytes, void* stream) {
   int rc = check_shape(B, H, N, d, dtype);
   if (rc) return rc;
   if ((rc = check_kv_heads(H, Hkv))) return rc;
   if ((rc = check_window(window_left, window_right))) return rc;
+  if ((rc = check_mask(mask, mask_heads, H, N, dtype))) return rc;
   if ((rc = check_scale(scale))) return rc;
   if (dtype != FA_BF16 || d != 128) return FA_ERR_UNSUPPORTED;
   if (static_cast<long long>(B) * H * N == 0) return FA_OK;
@@ -408,6 +451,9 @@ int fa_bwd_window(const void* Q, const void* K, const void* V, const void* O, co
   a.scale = scale;
   a.scale_log2 = scale * 1.4426950408889634f;
   set_window(window_left, window_right, &a.wl, &a.wr, &a.causal);
+  a.block_mask = mask;
+  a.mask_heads = mask_heads;
+  a.nb = (N + 127) / 128;
   a.O = O;
   a.dO = dO;
   a.LSE = LSE;
@@ -440,6 +486,26 @@ int fa_bwd_window(const void* Q, const void* K, const void* V, const void* O, co
   return FA_OK;
 }
 
+}  // namespace
+
+extern "C" {
+
+int fa_bwd_window(const void* Q, const void* K, const void* V, const void* O, const void* dO, const float* LSE,
+                  void* dQ, void* dK, void* dV, int B, int H, int Hkv, int N, int d, float scale, int window_left,
+                  int window_right, int dtype, void* workspace, size_t workspace_bytes, void* stream) {
+  return bwd_common(Q, K, V, O, dO, LSE, dQ, dK, dV, B, H, Hkv, N, d, scale, window_left, window_right, nullptr, 0,
+                    dtype, workspace, workspace_bytes, stream);
+}
+
+int fa_bwd_blocksparse(const void* Q, const void* K, const void* V, const void* O, const void* dO, const float* LSE,
+                       void* dQ, void* dK, void* dV, int B, int H, int Hkv, int N, int d, float scale,
+                       int window_left, int window_right, const void* block_mask, int mask_heads, int dtype,
+                       void* workspace, size_t workspace_bytes, void* stream) {
+  if (!block_mask && static_cast<long long>(B) * H * N > 0) return FA_ERR_INVALID_ARG;
+  return bwd_common(Q, K, V, O, dO, LSE, dQ, dK, dV, B, H, Hkv, N, d, scale, window_left, window_right,
+                    static_cast<const uint8_t*>(block_mask), mask_heads, dtype, workspace, workspace_bytes, stream);
+}
+
 int fa_bwd_gqa(const void* Q, const void* K, const void* V, const void* O, const void* dO, const float* LSE,
                void* dQ, void* dK, void* dV, int B, int H, int Hkv, int N, int d, float scale, int causal, int dtype,
                void* workspace, size_t workspace_bytes, void* stream) {
@@ -452,6 +518,49 @@ int fa_bwd(const void* Q, const void* K, const void* V, const void* O, const voi
            size_t workspace_bytes, void* stream) {
   return fa_bwd_window(Q, K, V, O, dO, LSE, dQ, dK, dV, B, H, H, N, d, scale, -1, causal ? 0 : -1, dtype,
                        workspace, workspace_bytes, stream);
+}
+
+int fa_merge_partial(float* O_acc, float* LSE_acc, const void* O_part, const float* LSE_part, void* O_out, int B,
+                     int H, int N, int d, int init, void* stream) {
+  int rc = check_shape(B, H, N, d, FA_BF16);
+  if (rc) return rc;
+  if (static_cast<long long>(B) * H * N == 0) return FA_OK;
+  if (!O_acc || !LSE_acc || !O_part || !LSE_part) return FA_ERR_INVALID_ARG;
+  if (!aligned16(O_acc) || !aligned16(O_part) || (O_out && !aligned16(O_out)) ||
+      (reinterpret_cast<uintptr_t>(LSE_acc) & 3u) || (reinterpret_cast<uintptr_t>(LSE_part) & 3u))
+    return FA_ERR_MISALIGNED;
+  DeviceState* st = nullptr;
+  if ((rc = device_state(&st))) return rc;
+  cudaError_t e = launch_merge(O_acc, LSE_acc, O_part, LSE_part, O_out, B, H, N, d, init ? 1 : 0,
+                               static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail_cuda(e);
+  return FA_OK;
+}
+
+int fa_accumulate_bf16(float* acc, const void* part, long long n, int init, void* stream) {
+  if (n < 0 || n % 8 != 0) return FA_ERR_INVALID_ARG;
+  if (n == 0) return FA_OK;
+  if (!acc || !part) return FA_ERR_INVALID_ARG;
+  if (!aligned16(acc) || !aligned16(part)) return FA_ERR_MISALIGNED;
+  DeviceState* st = nullptr;
+  int rc = device_state(&st);
+  if (rc) return rc;
+  cudaError_t e = launch_accumulate(acc, part, n, init ? 1 : 0, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail_cuda(e);
+  return FA_OK;
+}
+
+int fa_cast_bf16(void* out, const float* in, long long n, void* stream) {
+  if (n < 0 || n % 8 != 0) return FA_ERR_INVALID_ARG;
+  if (n == 0) return FA_OK;
+  if (!out || !in) return FA_ERR_INVALID_ARG;
+  if (!aligned16(out) || !aligned16(in)) return FA_ERR_MISALIGNED;
+  DeviceState* st = nullptr;
+  int rc = device_state(&st);
+  if (rc) return rc;
+  cudaError_t e = launch_cast(out, in, n, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail_cuda(e);
+  return FA_OK;
 }
 
 int fa_debug_umma(const void* A, const void* B, float* D, int N, int K, int a_mn_major, int b_mn_major, int a_tmem,

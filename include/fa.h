@@ -111,6 +111,26 @@ int fa_fwd_window(const void* Q, const void* K, const void* V, void* O, float* L
                   int d, float scale, int window_left, int window_right, int dtype, void* stream);
 
 /*
+ * Forward pass with a block-sparse mask ("Flash Attention" (Ultralytics
+ * glossary), "Flash Attention и смежные понятия": sparse attention scores only
+ * chosen query/key pairs; the block-sparse form skips empty blocks).
+ *   block_mask  device array of bytes [mask_heads][nb][nb], nb = ceil(N / 128):
+ *               query block i (rows 128 i .. 128 i + 127) sees key block j of
+ *               query head h when block_mask[(mh * nb + i) * nb + j] != 0, with
+ *               mh = 0 if mask_heads == 1 (one mask for every head), else h.
+ *               Shared by every batch entry.  Must not be null.
+ *   mask_heads  1 or H (FA_ERR_INVALID_ARG otherwise).
+ *   window_left, window_right  as fa_fwd_window; both masks apply.
+ * Key blocks a query block does not see are neither loaded nor multiplied.  A
+ * row that sees no key gets O = 0 and LSE = -inf.  bf16 only
+ * (FA_ERR_UNSUPPORTED for FA_FP32); nb <= 4096, i.e. N <= 524288
+ * (FA_ERR_TOO_LARGE otherwise).  Other arguments as fa_fwd_window.
+ */
+int fa_fwd_blocksparse(const void* Q, const void* K, const void* V, void* O, float* LSE, int B, int H, int Hkv,
+                       int N, int d, float scale, int window_left, int window_right, const void* block_mask,
+                       int mask_heads, int dtype, void* stream);
+
+/*
  * Forward pass with 8-bit inputs (FP8 attention as FlashAttention-3 runs it:
  * "Flash Attention" (karlkratz.de), "Versionen").
  *   Q        [B, N, H, d] e4m3 codes (one byte each); the value is scale_q * code.
@@ -183,6 +203,17 @@ int fa_bwd_window(const void* Q, const void* K, const void* V, const void* O, co
                   int window_right, int dtype, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Backward pass under the block-sparse mask of fa_fwd_blocksparse (same mask,
+ * window and heads as the forward that produced O and LSE).  Each key block
+ * visits only the query blocks that see it; a key that no query sees gets
+ * dK = dV = 0.  Other arguments, results and errors as fa_bwd_window.
+ */
+int fa_bwd_blocksparse(const void* Q, const void* K, const void* V, const void* O, const void* dO,
+                       const float* LSE, void* dQ, void* dK, void* dV, int B, int H, int Hkv, int N, int d,
+                       float scale, int window_left, int window_right, const void* block_mask, int mask_heads,
+                       int dtype, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * fa_bwd for callers that cannot allocate device memory when they run the
  * backward pass (runtimes whose device memory is laid out once at start-up,
  * or code that must not call cudaMalloc mid-run because it can synchronise
@@ -203,6 +234,40 @@ int fa_bwd_window(const void* Q, const void* K, const void* V, const void* O, co
 int fa_bwd_static_scratch(const void* Q, const void* K, const void* V, const void* O, const void* dO,
                           const float* LSE, void* dQ, void* dK, void* dV, int B, int H, int N, int d, float scale,
                           int causal, int dtype, void* stream);
+
+/*
+ * Helpers for attention over a sequence split into chunks, as ring attention
+ * runs it ("Flash Attention" (Ultralytics glossary), "Flash Attention и
+ * смежные понятия": each device computes blockwise attention for its part of
+ * the sequence while the key/value blocks travel around a ring of devices).
+ *
+ * fa_merge_partial: combine a query chunk's running result with the partial
+ * result of one more key chunk.  Each partial is exact attention over its keys
+ * (as fa_fwd returns it), so with m = max(LSE_acc, LSE_part) and
+ * w_x = exp(LSE_x - m):
+ *     O_acc = (w_acc O_acc + w_part O_part) / (w_acc + w_part),
+ *     LSE_acc = m + ln(w_acc + w_part)
+ * (the online softmax's correction between key blocks, "Flash Attention"
+ * (karlkratz.de), "Tiling").  A row where both sides saw no key stays O = 0,
+ * LSE = -inf.
+ *   O_acc     [B, N, H, d] fp32, in/out;  LSE_acc [B, H, N] fp32, in/out.
+ *   O_part    [B, N, H, d] bf16;          LSE_part [B, H, N] fp32.
+ *   O_out     [B, N, H, d] bf16 copy of the merged O, or NULL.
+ *   init      nonzero: O_acc, LSE_acc := the partial (their old contents unread).
+ *   d         64 or 128.
+ */
+int fa_merge_partial(float* O_acc, float* LSE_acc, const void* O_part, const float* LSE_part, void* O_out, int B,
+                     int H, int N, int d, int init, void* stream);
+
+/*
+ * acc[i] += part[i] (fp32 += bf16) for i < n, or acc[i] = part[i] when init is
+ * nonzero: the fp32 sum of one chunk's gradient contributions.  n a multiple
+ * of 8, both pointers 16-byte aligned.
+ */
+int fa_accumulate_bf16(float* acc, const void* part, long long n, int init, void* stream);
+
+/* out[i] = bf16(in[i]) (round to nearest even) for i < n; n a multiple of 8. */
+int fa_cast_bf16(void* out, const float* in, long long n, void* stream);
 
 /* Static English text for a status code. */
 const char* fa_status_string(int status);
