@@ -211,6 +211,18 @@ CUresult make_tile_map_e4m3(CUtensorMap* map, const void* base, int B, int N, in
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
 }
 
+CUresult make_dq_accum_map_sw128(CUtensorMap* map, float* base, int B, int N, int H, int d) {
+  if (!encoder()) return CUDA_ERROR_NOT_FOUND;
+  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(H),
+                              static_cast<cuuint64_t>(B)};
+  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(H) * d * 4, static_cast<cuuint64_t>(d) * 4,
+                                 static_cast<cuuint64_t>(N) * H * d * 4};
+  const cuuint32_t box[4] = {32u, 128u, 1u, 1u};
+  const cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+  return g_encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+}
+
 CUresult make_dq_accum_map(CUtensorMap* map, float* base, int B, int N, int H, int d) {
   if (!encoder()) return CUDA_ERROR_NOT_FOUND;
   const cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(H),
@@ -428,7 +440,7 @@ int bwd_common(const void* Q, const void* K, const void* V, const void* O, const
   if ((rc = check_window(window_left, window_right))) return rc;
   if ((rc = check_mask(mask, mask_heads, H, N, dtype))) return rc;
   if ((rc = check_scale(scale))) return rc;
-  if (dtype != FA_BF16 || d != 128) return FA_ERR_UNSUPPORTED;
+  if (dtype != FA_BF16) return FA_ERR_UNSUPPORTED;
   if (static_cast<long long>(B) * H * N == 0) return FA_OK;
   if (!Q || !K || !V || !O || !dO || !LSE || !dQ || !dK || !dV) return FA_ERR_INVALID_ARG;
   const void* ptrs[] = {Q, K, V, O, dO, LSE, dQ, dK, dV};
@@ -473,12 +485,14 @@ int bwd_common(const void* Q, const void* K, const void* V, const void* O, const
       (r = make_tile_map(&tdo, dO, B, N, H, d, 128)) != CUDA_SUCCESS ||
       (r = make_tile_map(&tk, K, B, N, Hkv, d, 128)) != CUDA_SUCCESS ||
       (r = make_tile_map(&tv, V, B, N, Hkv, d, 128)) != CUDA_SUCCESS ||
-      (r = make_dq_accum_map(&tdq, a.dQacc, B, N, H, d)) != CUDA_SUCCESS)
+      (r = (d == 128 ? make_dq_accum_map(&tdq, a.dQacc, B, N, H, d)
+                     : make_dq_accum_map_sw128(&tdq, a.dQacc, B, N, H, d))) != CUDA_SUCCESS)
     return fail_encode(r);
   cudaError_t e = launch_bwd_pre(a, s);
   if (e != cudaSuccess) return fail_cuda(e);
   if (t_ev_start) cudaEventRecord(t_ev_start, s);
-  e = launch_bwd_main(tq, tk, tv, tdo, tdq, a, make_ctl(*st), s);
+  e = (d == 128) ? launch_bwd_main(tq, tk, tv, tdo, tdq, a, make_ctl(*st), s)
+                 : launch_bwd_main64(tq, tk, tv, tdo, tdq, a, make_ctl(*st), s);
   if (e != cudaSuccess) return fail_cuda(e);
   if (t_ev_stop) cudaEventRecord(t_ev_stop, s);
   e = launch_bwd_dq(a, s);

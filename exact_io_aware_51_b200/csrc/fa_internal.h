@@ -73,6 +73,10 @@ CUresult make_tile_map_e4m3(CUtensorMap* map, const void* base, int B, int N, in
 // sequence positions x d features of one (b, h), no swizzle (for TMA reduce-add).
 CUresult make_dq_accum_map(CUtensorMap* map, float* base, int B, int N, int H, int d);
 
+// TMA descriptor for the fp32 dQ accumulator as the d = 64 backward adds into it:
+// a box of 32 features x 128 sequence positions of one (b, h), 128-byte swizzle.
+CUresult make_dq_accum_map_sw128(CUtensorMap* map, float* base, int B, int N, int H, int d);
+
 // Kernel launchers (each returns the cudaError_t of the launch).
 cudaError_t launch_fwd_bf16(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const FwdArgs& a, const DevCtl& c, cudaStream_t s);
@@ -83,6 +87,9 @@ cudaError_t launch_bwd_pre(const BwdArgs& a, cudaStream_t s);
 cudaError_t launch_bwd_main(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const CUtensorMap& tdo, const CUtensorMap& tdq, const BwdArgs& a, const DevCtl& c,
                             cudaStream_t s);
+cudaError_t launch_bwd_main64(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                              const CUtensorMap& tdo, const CUtensorMap& tdq, const BwdArgs& a, const DevCtl& c,
+                              cudaStream_t s);
 cudaError_t launch_bwd_dq(const BwdArgs& a, cudaStream_t s);
 
 // Chunked-sequence (ring) helpers: merge of partial results, fp32 accumulation, cast.

@@ -169,7 +169,7 @@ size_t fa_bwd_workspace_size(int B, int H, int N, int d, int dtype);
  *   dQ, dK, dV      [B, N, H, d] outputs, written completely.
  *   workspace       device buffer of at least fa_bwd_workspace_size() bytes,
  *                   256-byte aligned; overwritten.
- * Currently dtype FA_BF16 with d = 128 (FA_ERR_UNSUPPORTED otherwise).
+ * dtype FA_BF16 with d = 64 or 128 (FA_ERR_UNSUPPORTED for FA_FP32).
  * dQ is summed over key tiles by fp32 reduce-adds in L2 whose order varies
  * from run to run, so it is not bitwise deterministic.
  */

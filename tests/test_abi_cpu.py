@@ -76,9 +76,13 @@ def test_backward_validation(L):
     b = L.fa_bwd
     args = [16] * 9
     ws = L.fa_bwd_workspace_size(1, 1, 128, 128, 0)
-    # fp32 backward and d = 64 backward are not implemented: refused
+    # the fp32 backward is not implemented: refused
     assert b(*args, 1, 1, 128, 128, 0.1, 0, 1, 256, ws, None) == -2
-    assert b(*args, 1, 1, 128, 64, 0.1, 0, 0, 256, ws, None) == -2
+    # d = 64 passes the dtype / head-dim check and reaches the alignment check
+    bad64 = list(args)
+    bad64[3] = 24
+    ws64 = L.fa_bwd_workspace_size(1, 1, 128, 64, 0)
+    assert b(*bad64, 1, 1, 128, 64, 0.1, 0, 0, 256, ws64, None) == -3
     # workspace missing / too small / misaligned
     assert b(*args, 1, 1, 128, 128, 0.1, 0, 0, None, ws, None) == -4
     assert b(*args, 1, 1, 128, 128, 0.1, 0, 0, 256, ws - 1, None) == -4
