@@ -37,7 +37,7 @@ EXPORTED = ("fa_fwd", "fa_bwd_workspace_size", "fa_bwd", "fa_status_string", "fa
             "fa_version", "fa_set_kernel_events", "fa_bwd_static_scratch", "fa_fwd_gqa", "fa_bwd_gqa",
             "fa_fwd_window", "fa_bwd_window", "fa_debug_umma_f8", "fa_fwd_fp8",
             "fa_fwd_blocksparse", "fa_bwd_blocksparse", "fa_merge_partial", "fa_accumulate_bf16",
-            "fa_cast_bf16")
+            "fa_cast_bf16", "fa_bwd_workspace_size_gqa")
 
 
 class FAError(RuntimeError):
@@ -69,6 +69,8 @@ def lib() -> ctypes.CDLL:
     L.fa_fwd.restype = i
     L.fa_bwd_workspace_size.argtypes = [i, i, i, i, i]
     L.fa_bwd_workspace_size.restype = sz
+    L.fa_bwd_workspace_size_gqa.argtypes = [i, i, i, i, i, i]
+    L.fa_bwd_workspace_size_gqa.restype = sz
     L.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, i, vp, sz, vp]
     L.fa_bwd.restype = i
     L.fa_fwd_gqa.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp]
@@ -273,8 +275,11 @@ def cast_bf16(x, out=None, stream=None):
     return out
 
 
-def bwd_workspace_size(B: int, H: int, N: int, d: int, dtype: int = FA_BF16) -> int:
-    return int(lib().fa_bwd_workspace_size(B, H, N, d, dtype))
+def bwd_workspace_size(B: int, H: int, N: int, d: int, dtype: int = FA_BF16, kv_heads: int | None = None) -> int:
+    """Backward workspace bytes (with the split accumulators small problems use)."""
+    if kv_heads is None:
+        return int(lib().fa_bwd_workspace_size(B, H, N, d, dtype))
+    return int(lib().fa_bwd_workspace_size_gqa(B, H, kv_heads, N, d, dtype))
 
 
 def bwd(q, k, v, o, do, lse, causal: bool = False, scale: float | None = None, workspace=None,
@@ -292,7 +297,7 @@ def bwd(q, k, v, o, do, lse, causal: bool = False, scale: float | None = None, w
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
-    need = bwd_workspace_size(B, H, N, d, _dtype_code(q))
+    need = bwd_workspace_size(B, H, N, d, _dtype_code(q), kv_heads=Hkv)
     if workspace is None:
         workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
     ptrs = (q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(), lse.data_ptr(),

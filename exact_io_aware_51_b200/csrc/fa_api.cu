@@ -163,6 +163,37 @@ void set_window(int left, int right, int* wl, int* wr, int* causal) {
   *causal = (*wl == kUnbounded && *wr == 0) ? 1 : 0;
 }
 
+// Parts each key tile's (query head, query tile) walk is split into (1, 2, 4 or
+// 8; each part keeps at least 8 query tiles, non-causal count).  One CTA runs
+// per SM (148 SMs).
+//   * Unmasked walks are equally long: the launch takes ceil(CTAs / 148) waves
+//     of whole walks, so parts = p costs ceil(p CTAs / 148) / p waves, plus the
+//     partial sums (zeroing, reduce-adds, convert), taken as the time of 4 query
+//     tiles per part: a factor 1 + 4 p / (query tiles per walk).  The cheapest p
+//     wins (ties: fewer parts).  Measured on B200: +16% at B1 H64 Hkv8 N8192
+//     d128 (2 parts), and the factor keeps d = 64 walks of 32 tiles unsplit.
+//   * Causal and windowed walks differ in length from one key tile to the next,
+//     so a grid of fewer than three waves is split until it has three.
+int bwd_splits(int B, int H, int Hkv, int N, bool masked) {
+  const long long nkt = (static_cast<long long>(N) + 127) / 128;
+  const long long ctas = nkt * Hkv * B;
+  const long long per_cta = (H / (Hkv > 0 ? Hkv : 1)) * nkt;
+  int parts = 1;
+  if (masked) {
+    while (parts < 8 && ctas * parts < 3 * 148 && per_cta / (2 * parts) >= 8) parts *= 2;
+    return parts;
+  }
+  double best = static_cast<double>((ctas + 147) / 148);
+  for (int p = 2; p <= 8 && per_cta / p >= 8; p *= 2) {
+    const double cost = static_cast<double>((ctas * p + 147) / 148) / p * (1.0 + 4.0 * p / per_cta);
+    if (cost < best - 1e-9) {
+      best = cost;
+      parts = p;
+    }
+  }
+  return parts;
+}
+
 int check_scale(float scale) {
   if (!std::isfinite(scale) || !(scale > 0.f)) return FA_ERR_INVALID_ARG;
   return FA_OK;
@@ -209,6 +240,27 @@ CUresult make_tile_map_e4m3(CUtensorMap* map, const void* base, int B, int N, in
   return g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void*>(base), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+}
+
+size_t bwd_workspace_base(int B, int H, int N, int d, int dtype) {
+  if (check_shape(B, H, N, d, dtype) != FA_OK) return 0;
+  if (static_cast<long long>(B) * H * N == 0) return 0;
+  const size_t npad = (static_cast<size_t>(N) + 127) / 128 * 128;
+  const size_t dq = align256(static_cast<size_t>(B) * N * H * d * sizeof(float));
+  const size_t rows = align256(static_cast<size_t>(B) * H * npad * sizeof(float));
+  return dq + 2 * rows;
+}
+
+CUresult make_kv_accum_map(CUtensorMap* map, float* base, int B, int N, int Hkv, int d) {
+  if (!encoder()) return CUDA_ERROR_NOT_FOUND;
+  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(Hkv),
+                              static_cast<cuuint64_t>(B)};
+  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(Hkv) * d * 4, static_cast<cuuint64_t>(d) * 4,
+                                 static_cast<cuuint64_t>(N) * Hkv * d * 4};
+  const cuuint32_t box[4] = {static_cast<cuuint32_t>(d), d == 128 ? 64u : 128u, 1u, 1u};
+  const cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+  return g_encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
 }
 
 CUresult make_dq_accum_map_sw128(CUtensorMap* map, float* base, int B, int N, int H, int d) {
@@ -418,13 +470,18 @@ int fa_fwd_fp8(const void* Q, const void* K, const void* V, void* O, float* LSE,
   return FA_OK;
 }
 
+size_t fa_bwd_workspace_size_gqa(int B, int H, int Hkv, int N, int d, int dtype) {
+  if (check_kv_heads(H, Hkv) != FA_OK) return 0;
+  const size_t base = fa::bwd_workspace_base(B, H, N, d, dtype);
+  if (base == 0) return 0;
+  // the accumulators whenever masked or unmasked walks of this shape would split
+  const bool split = bwd_splits(B, H, Hkv, N, true) > 1 || bwd_splits(B, H, Hkv, N, false) > 1;
+  const size_t kv = split ? 2 * align256(static_cast<size_t>(B) * N * Hkv * d * sizeof(float)) : 0;
+  return base + kv;
+}
+
 size_t fa_bwd_workspace_size(int B, int H, int N, int d, int dtype) {
-  if (check_shape(B, H, N, d, dtype) != FA_OK) return 0;
-  if (static_cast<long long>(B) * H * N == 0) return 0;
-  const size_t npad = (static_cast<size_t>(N) + 127) / 128 * 128;
-  const size_t dq = align256(static_cast<size_t>(B) * N * H * d * sizeof(float));
-  const size_t rows = align256(static_cast<size_t>(B) * H * npad * sizeof(float));
-  return dq + 2 * rows;
+  return fa_bwd_workspace_size_gqa(B, H, H, N, d, dtype);
 }
 
 }  // extern "C"
@@ -446,8 +503,13 @@ int bwd_common(const void* Q, const void* K, const void* V, const void* O, const
   const void* ptrs[] = {Q, K, V, O, dO, LSE, dQ, dK, dV};
   for (const void* p : ptrs)
     if (!aligned16(p)) return FA_ERR_MISALIGNED;
-  const size_t need = fa_bwd_workspace_size(B, H, N, d, dtype);
+  const size_t need = bwd_workspace_base(B, H, N, d, dtype);
   if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return FA_ERR_WORKSPACE;
+  // split the walks when the grid is small and the workspace holds the fp32 dK / dV sums
+  const bool masked = window_left >= 0 || window_right >= 0 || mask != nullptr;
+  const int parts = (workspace_bytes >= fa_bwd_workspace_size_gqa(B, H, Hkv, N, d, dtype))
+                        ? bwd_splits(B, H, Hkv, N, masked)
+                        : 1;
   DeviceState* st = nullptr;
   if ((rc = device_state(&st))) return rc;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -478,8 +540,13 @@ int bwd_common(const void* Q, const void* K, const void* V, const void* O, const
   a.Dvec = reinterpret_cast<float*>(ws);
   ws += align256(static_cast<size_t>(B) * H * npad * sizeof(float));
   a.LSE2 = reinterpret_cast<float*>(ws);
+  ws += align256(static_cast<size_t>(B) * H * npad * sizeof(float));
+  a.splits = parts;
+  a.dKacc = parts > 1 ? reinterpret_cast<float*>(ws) : nullptr;
+  a.dVacc = parts > 1 ? reinterpret_cast<float*>(ws + align256(static_cast<size_t>(B) * N * Hkv * d * sizeof(float)))
+                      : nullptr;
 
-  CUtensorMap tq, tk, tv, tdo, tdq;
+  CUtensorMap tq, tk, tv, tdo, tdq, tdk, tdv;
   CUresult r;
   if ((r = make_tile_map(&tq, Q, B, N, H, d, 128)) != CUDA_SUCCESS ||
       (r = make_tile_map(&tdo, dO, B, N, H, d, 128)) != CUDA_SUCCESS ||
@@ -488,14 +555,24 @@ int bwd_common(const void* Q, const void* K, const void* V, const void* O, const
       (r = (d == 128 ? make_dq_accum_map(&tdq, a.dQacc, B, N, H, d)
                      : make_dq_accum_map_sw128(&tdq, a.dQacc, B, N, H, d))) != CUDA_SUCCESS)
     return fail_encode(r);
+  if (parts > 1) {
+    if ((r = make_kv_accum_map(&tdk, a.dKacc, B, N, Hkv, d)) != CUDA_SUCCESS ||
+        (r = make_kv_accum_map(&tdv, a.dVacc, B, N, Hkv, d)) != CUDA_SUCCESS)
+      return fail_encode(r);
+  } else {
+    tdk = tdq;  // not read by the kernels without a split
+    tdv = tdq;
+  }
   cudaError_t e = launch_bwd_pre(a, s);
+  if (e == cudaSuccess && parts > 1) e = launch_bwd_kv_zero(a, s);
   if (e != cudaSuccess) return fail_cuda(e);
   if (t_ev_start) cudaEventRecord(t_ev_start, s);
-  e = (d == 128) ? launch_bwd_main(tq, tk, tv, tdo, tdq, a, make_ctl(*st), s)
-                 : launch_bwd_main64(tq, tk, tv, tdo, tdq, a, make_ctl(*st), s);
+  e = (d == 128) ? launch_bwd_main(tq, tk, tv, tdo, tdq, tdk, tdv, a, make_ctl(*st), s)
+                 : launch_bwd_main64(tq, tk, tv, tdo, tdq, tdk, tdv, a, make_ctl(*st), s);
   if (e != cudaSuccess) return fail_cuda(e);
   if (t_ev_stop) cudaEventRecord(t_ev_stop, s);
   e = launch_bwd_dq(a, s);
+  if (e == cudaSuccess && parts > 1) e = launch_bwd_kv_convert(a, s);
   if (e != cudaSuccess) return fail_cuda(e);
   return FA_OK;
 }

@@ -154,6 +154,7 @@ struct BwdBars {
   // their q_full wait)
   int info_q0[4];
   int sparse_nq;  // block-sparse: kept (query head, query tile) pairs of this key tile
+  uint64_t epi_sync[2];  // split walks: a compute warpgroup's partial dV / dK is staged
 };
 static_assert(sizeof(BwdBars) <= 256, "barrier block");
 static_assert(BwdCfg::kOffDQS % 1024 == 0 && BwdCfg::kSmemBytes <= 232448, "shared memory layout");
@@ -189,7 +190,8 @@ template <bool kSparse>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
-                    const __grid_constant__ CUtensorMap tmDQ, const BwdArgs a, const DevCtl ctl) {
+                    const __grid_constant__ CUtensorMap tmDQ, const __grid_constant__ CUtensorMap tmDK,
+                    const __grid_constant__ CUtensorMap tmDV, const BwdArgs a, const DevCtl ctl) {
   using C = BwdCfg;
   constexpr int D = C::D;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -202,8 +204,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = warp_id();
   const int lane = lane_id();
 
-  const int jt = blockIdx.x;  // key tile
-  const int hk = blockIdx.y;  // K/V head
+  const int jt = blockIdx.x;                // key tile
+  const int hk = blockIdx.y / a.splits;     // K/V head
+  const int sp = blockIdx.y % a.splits;     // part of this key tile's walk
   const int b = blockIdx.z;
   const int key0 = jt * kBN;
   const int nq_total = (a.N + kBMq - 1) / kBMq;
@@ -240,8 +243,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     nq = s_nq;
   }
+  // split walks: this CTA takes iterations [beg, beg + nq) of the key tile's walk
+  const int beg = static_cast<int>((static_cast<long long>(nq) * sp) / a.splits);
+  nq = static_cast<int>((static_cast<long long>(nq) * (sp + 1)) / a.splits) - beg;
+  const int qt_beg = (nq_head > 0) ? i0 + beg % nq_head : i0;     // dense walk: first query tile
+  const int hq_beg = hk * G + ((nq_head > 0) ? beg / nq_head : 0);  // and its query head
 
   if (threadIdx.x == 0) {
+    mbar_init(&bars->epi_sync[0], 128);
+    mbar_init(&bars->epi_sync[1], 128);
     mbar_init(&bars->kv_full, 1);
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&bars->q_full[s], 1);
@@ -280,7 +290,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t tR2 = tmem + lane_bits + C::kColR2 + 64 * g;
       const float sl2 = a.scale_log2;
       bool ok = true;
-      int qt = i0;  // query tile of iteration i (the head does not matter here)
+      int qt = qt_beg;  // query tile of iteration i (the head does not matter here)
       for (int i = 0; i < nq; ++i) {
         const int st = i % kStages;
         const uint32_t par = i & 1;
@@ -383,7 +393,39 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // ---- epilogue: WG0 writes the dV rows, WG1 the dK rows of its keys ----
       if (ok && nq > 0) ok = warp_all(wait_bar(&bars->acc_done, 0, w, 23));
-      if (ok) {
+      if (ok && a.splits > 1) {
+        // a part of a split walk: add the fp32 partial sums into the accumulator.
+        // The Q (WG0) or dO (WG1) stages, idle now, hold the [128 keys][128] fp32
+        // rows; two TMA reduce-adds of 64 keys each carry them to global memory.
+        tc_fence_after();
+        float* stg = reinterpret_cast<float*>(smem + (g == 0 ? C::kOffQ : C::kOffDO));
+        const uint32_t col = g == 0 ? C::kColDV : C::kColDK;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t v[32];
+          if (nq > 0) {
+            tmem_ld32(tmem + lane_bits + col + c * 32, v);
+            tmem_wait_ld();
+            reg_fence32(v);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = 0u;
+          }
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            st_shared_v4(smem_u32(stg + r * D + c * 32 + 4 * i), v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(&bars->epi_sync[g]);
+        ok = warp_all(wait_bar(&bars->epi_sync[g], 0, w, 25));
+        if (ok && r == 0) {
+          const CUtensorMap* m = g == 0 ? &tmDV : &tmDK;
+          tma_reduce_add_4d(m, stg, 0, key0, hk, b);
+          tma_reduce_add_4d(m, stg + 64 * D, 0, key0 + 64, hk, b);
+          bulk_commit();
+          bulk_wait_all();
+        }
+      } else if (ok) {
         tc_fence_after();
         const size_t base = ((static_cast<size_t>(b) * a.N + key) * a.Hkv + hk) * D;
         const uint32_t col = g == 0 ? C::kColDV : C::kColDK;
@@ -434,12 +476,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++sync_phase;
         return r;
       };
-      int qt = i0, hq = hk * G;
+      int qt = qt_beg, hq = hq_beg;
       if constexpr (kSparse) {
-        while (hq < hk * G + G && !kept(hq, qt)) {
-          if (++qt == qt_end) {
+        // the first kept pair, then past the `beg` kept pairs of the earlier parts
+        qt = i0;
+        hq = hk * G;
+        for (int skip = -1; skip < beg; ++skip) {
+          if (skip >= 0 && ++qt == qt_end) {
             qt = i0;
             ++hq;
+          }
+          while (hq < hk * G + G && !kept(hq, qt)) {
+            if (++qt == qt_end) {
+              qt = i0;
+              ++hq;
+            }
           }
         }
       }
@@ -491,12 +542,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_4d(smem + C::kOffK + c * C::kSub, &tmK, &bars->kv_full, c * 64, key0, hk, b);
           tma_load_4d(smem + C::kOffV + c * C::kSub, &tmV, &bars->kv_full, c * 64, key0, hk, b);
         }
-        int qt = i0, hq = hk * G;
+        int qt = qt_beg, hq = hq_beg;
         if constexpr (kSparse) {
-          while (hq < hk * G + G && !kept(hq, qt)) {
-            if (++qt == qt_end) {
+          // the first kept pair, then past the `beg` kept pairs of the earlier parts
+          qt = i0;
+          hq = hk * G;
+          for (int skip = -1; skip < beg; ++skip) {
+            if (skip >= 0 && ++qt == qt_end) {
               qt = i0;
               ++hq;
+            }
+            while (hq < hk * G + G && !kept(hq, qt)) {
+              if (++qt == qt_end) {
+                qt = i0;
+                ++hq;
+              }
             }
           }
         }
@@ -623,17 +683,64 @@ cudaError_t launch_bwd_pre(const BwdArgs& a, cudaStream_t s) {
 }
 
 cudaError_t launch_bwd_main(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                            const CUtensorMap& tdo, const CUtensorMap& tdq, const BwdArgs& a, const DevCtl& c,
-                            cudaStream_t s) {
+                            const CUtensorMap& tdo, const CUtensorMap& tdq, const CUtensorMap& tdk,
+                            const CUtensorMap& tdv, const BwdArgs& a, const DevCtl& c, cudaStream_t s) {
   constexpr int smem = BwdCfg::kSmemBytes;
-  const dim3 grid((a.N + kBN - 1) / kBN, a.Hkv, a.B);
+  const dim3 grid((a.N + kBN - 1) / kBN, a.Hkv * a.splits, a.B);
   auto run = [&](auto kernel) -> cudaError_t {
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    kernel<<<grid, kThreads, smem, s>>>(tq, tk, tv, tdo, tdq, a, c);
+    kernel<<<grid, kThreads, smem, s>>>(tq, tk, tv, tdo, tdq, tdk, tdv, a, c);
     return cudaGetLastError();
   };
   return a.block_mask ? run(bwd_main_kernel<true>) : run(bwd_main_kernel<false>);
+}
+
+namespace {
+__global__ void __launch_bounds__(256) kv_zero_kernel(float* __restrict__ p, long long n4) {
+  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4;
+       i += static_cast<long long>(gridDim.x) * blockDim.x)
+    reinterpret_cast<float4*>(p)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+}
+
+// dK = bf16(scale * dKacc), dV = bf16(dVacc), 8 elements per thread
+__global__ void __launch_bounds__(256) kv_convert_kernel(const BwdArgs a, long long total) {
+  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x * 8;
+  for (long long i = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) * 8; i < total; i += stride) {
+#pragma unroll
+    for (int which = 0; which < 2; ++which) {
+      const float* src = which ? a.dKacc : a.dVacc;
+      const float s = which ? a.scale : 1.f;
+      const float4 x = *reinterpret_cast<const float4*>(src + i);
+      const float4 y = *reinterpret_cast<const float4*>(src + i + 4);
+      uint4 out;
+      out.x = pack_bf16x2(x.x * s, x.y * s);
+      out.y = pack_bf16x2(x.z * s, x.w * s);
+      out.z = pack_bf16x2(y.x * s, y.y * s);
+      out.w = pack_bf16x2(y.z * s, y.w * s);
+      *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(which ? a.dK : a.dV) + i) = out;
+    }
+  }
+}
+
+unsigned blocks_for(long long items) {
+  long long blocks = (items + 255) / 256;
+  if (blocks > 148 * 16) blocks = 148 * 16;
+  return static_cast<unsigned>(blocks < 1 ? 1 : blocks);
+}
+}  // namespace
+
+cudaError_t launch_bwd_kv_zero(const BwdArgs& a, cudaStream_t s) {
+  const long long n = static_cast<long long>(a.B) * a.N * a.Hkv * a.d;  // per accumulator, a multiple of 64
+  kv_zero_kernel<<<blocks_for(n / 4), 256, 0, s>>>(a.dKacc, n / 4);
+  kv_zero_kernel<<<blocks_for(n / 4), 256, 0, s>>>(a.dVacc, n / 4);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bwd_kv_convert(const BwdArgs& a, cudaStream_t s) {
+  const long long total = static_cast<long long>(a.B) * a.N * a.Hkv * a.d;
+  kv_convert_kernel<<<blocks_for(total / 8), 256, 0, s>>>(a, total);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_bwd_dq(const BwdArgs& a, cudaStream_t s) {

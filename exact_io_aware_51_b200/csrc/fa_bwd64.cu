@@ -69,6 +69,7 @@ struct Bars {
   int abort;
   int info_q0[4];  // block-sparse: first query row of tile i in slot i % 4 (as at d = 128)
   int sparse_nq;
+  uint64_t epi_sync[2];  // split walks: a compute warpgroup's partial dV / dK is staged
 };
 static_assert(sizeof(Bars) <= 256, "barrier block");
 
@@ -101,7 +102,8 @@ template <bool kSparse>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd64_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
-                 const __grid_constant__ CUtensorMap tmDQ, const BwdArgs a, const DevCtl ctl) {
+                 const __grid_constant__ CUtensorMap tmDQ, const __grid_constant__ CUtensorMap tmDK,
+                 const __grid_constant__ CUtensorMap tmDV, const BwdArgs a, const DevCtl ctl) {
   using C = Cfg;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = smem_raw;
@@ -114,7 +116,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int lane = lane_id();
 
   const int jt = blockIdx.x;
-  const int hk = blockIdx.y;
+  const int hk = blockIdx.y / a.splits;
+  const int sp = blockIdx.y % a.splits;
   const int b = blockIdx.z;
   const int key0 = jt * kBN;
   const int nq_total = (a.N + kBMq - 1) / kBMq;
@@ -141,8 +144,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     nq = s_nq;
   }
+  const int beg = static_cast<int>((static_cast<long long>(nq) * sp) / a.splits);
+  nq = static_cast<int>((static_cast<long long>(nq) * (sp + 1)) / a.splits) - beg;
+  const int qt_beg = (nq_head > 0) ? i0 + beg % nq_head : i0;
+  const int hq_beg = hk * G + ((nq_head > 0) ? beg / nq_head : 0);
 
   if (threadIdx.x == 0) {
+    mbar_init(&bars->epi_sync[0], 128);
+    mbar_init(&bars->epi_sync[1], 128);
     mbar_init(&bars->kv_full, 1);
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&bars->q_full[s], 1);
@@ -181,7 +190,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t tR2 = tmem + lane_bits + C::kColR2 + 64 * g;
       const float sl2 = a.scale_log2;
       bool ok = true;
-      int qt = i0;
+      int qt = qt_beg;
       for (int i = 0; i < nq; ++i) {
         const int st = i % kStages;
         const uint32_t par = i & 1;
@@ -270,7 +279,36 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // ---- epilogue: WG0 writes the dV rows, WG1 the dK rows of its keys ----
       if (ok && nq > 0) ok = warp_all(wait_bar(&bars->acc_done, 0, w, 44));
-      if (ok) {
+      if (ok && a.splits > 1) {
+        // a part of a split walk: the Q (WG0) or dO (WG1) stages hold the
+        // [128 keys][64] fp32 partial sums for one TMA reduce-add
+        tc_fence_after();
+        float* stg = reinterpret_cast<float*>(smem + (g == 0 ? C::kOffQ : C::kOffDO));
+        const uint32_t col = g == 0 ? C::kColDV : C::kColDK;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t v[32];
+          if (nq > 0) {
+            tmem_ld32(tmem + lane_bits + col + c * 32, v);
+            tmem_wait_ld();
+            reg_fence32(v);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = 0u;
+          }
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            st_shared_v4(smem_u32(stg + r * D + c * 32 + 4 * i), v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(&bars->epi_sync[g]);
+        ok = warp_all(wait_bar(&bars->epi_sync[g], 0, w, 55));
+        if (ok && r == 0) {
+          tma_reduce_add_4d(g == 0 ? &tmDV : &tmDK, stg, 0, key0, hk, b);
+          bulk_commit();
+          bulk_wait_all();
+        }
+      } else if (ok) {
         tc_fence_after();
         const size_t base = ((static_cast<size_t>(b) * a.N + key) * a.Hkv + hk) * D;
         const uint32_t col = g == 0 ? C::kColDV : C::kColDK;
@@ -319,12 +357,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++sync_phase;
         return r;
       };
-      int qt = i0, hq = hk * G;
+      int qt = qt_beg, hq = hq_beg;
       if constexpr (kSparse) {
-        while (hq < hk * G + G && !kept(hq, qt)) {
-          if (++qt == qt_end) {
+        qt = i0;
+        hq = hk * G;
+        for (int skip = -1; skip < beg; ++skip) {
+          if (skip >= 0 && ++qt == qt_end) {
             qt = i0;
             ++hq;
+          }
+          while (hq < hk * G + G && !kept(hq, qt)) {
+            if (++qt == qt_end) {
+              qt = i0;
+              ++hq;
+            }
           }
         }
       }
@@ -378,12 +424,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive_expect_tx(&bars->kv_full, 2 * C::kTile);
         tma_load_4d(smem + C::kOffK, &tmK, &bars->kv_full, 0, key0, hk, b);
         tma_load_4d(smem + C::kOffV, &tmV, &bars->kv_full, 0, key0, hk, b);
-        int qt = i0, hq = hk * G;
+        int qt = qt_beg, hq = hq_beg;
         if constexpr (kSparse) {
-          while (hq < hk * G + G && !kept(hq, qt)) {
-            if (++qt == qt_end) {
+          qt = i0;
+          hq = hk * G;
+          for (int skip = -1; skip < beg; ++skip) {
+            if (skip >= 0 && ++qt == qt_end) {
               qt = i0;
               ++hq;
+            }
+            while (hq < hk * G + G && !kept(hq, qt)) {
+              if (++qt == qt_end) {
+                qt = i0;
+                ++hq;
+              }
             }
           }
         }
@@ -493,14 +547,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 }  // namespace
 
 cudaError_t launch_bwd_main64(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                              const CUtensorMap& tdo, const CUtensorMap& tdq, const BwdArgs& a, const DevCtl& c,
-                              cudaStream_t s) {
+                              const CUtensorMap& tdo, const CUtensorMap& tdq, const CUtensorMap& tdk,
+                              const CUtensorMap& tdv, const BwdArgs& a, const DevCtl& c, cudaStream_t s) {
   constexpr int smem = Cfg::kSmemBytes;
-  const dim3 grid((a.N + kBN - 1) / kBN, a.Hkv, a.B);
+  const dim3 grid((a.N + kBN - 1) / kBN, a.Hkv * a.splits, a.B);
   auto run = [&](auto kernel) -> cudaError_t {
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    kernel<<<grid, kThreads, smem, s>>>(tq, tk, tv, tdo, tdq, a, c);
+    kernel<<<grid, kThreads, smem, s>>>(tq, tk, tv, tdo, tdq, tdk, tdv, a, c);
     return cudaGetLastError();
   };
   return a.block_mask ? run(bwd64_kernel<true>) : run(bwd64_kernel<false>);

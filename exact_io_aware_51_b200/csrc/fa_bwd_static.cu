@@ -72,7 +72,7 @@ int scratch_address(void** out) {
 extern "C" int fa_bwd_static_scratch(const void* Q, const void* K, const void* V, const void* O, const void* dO,
                                      const float* LSE, void* dQ, void* dK, void* dV, int B, int H, int N, int d,
                                      float scale, int causal, int dtype, void* stream) {
-  const size_t need = fa_bwd_workspace_size(B, H, N, d, dtype);
+  const size_t need = fa::bwd_workspace_base(B, H, N, d, dtype);
   if (need > fa::kStaticScratchBytes) return FA_ERR_TOO_LARGE;
   if (need == 0) {
     // invalid or empty problem: fa_bwd reports which, without touching scratch

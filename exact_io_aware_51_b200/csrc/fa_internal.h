@@ -59,7 +59,17 @@ struct BwdArgs {
   float* LSE2;       // [B, H, Npad] LSE * log2(e)
   const uint8_t* block_mask;  // as in FwdArgs (nullptr: none)
   int mask_heads, nb;
+  // Split of each key tile's (query head, query tile) walk over `splits` CTAs
+  // (small grids): with splits > 1 the CTAs add their dK, dV partial sums into
+  // these fp32 [B, N, Hkv, d] accumulators (zeroed first) instead of writing dK, dV.
+  int splits;
+  float* dKacc;
+  float* dVacc;
 };
+
+// Bytes of backward workspace a call cannot do without (dQ accumulator and the two
+// per-row arrays); the public size functions may add the split accumulators.
+size_t bwd_workspace_base(int B, int H, int N, int d, int dtype);
 
 // TMA descriptor for a [B, N, H, d] bf16 tensor with a box of `rows` sequence
 // positions x 64 features of one (b, h); 128-byte swizzle.
@@ -85,11 +95,17 @@ cudaError_t launch_fwd_fp8(const CUtensorMap& tq, const CUtensorMap& tk, const C
 cudaError_t launch_fwd_f32(const float* Q, const float* K, const float* V, const FwdArgs& a, cudaStream_t s);
 cudaError_t launch_bwd_pre(const BwdArgs& a, cudaStream_t s);
 cudaError_t launch_bwd_main(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                            const CUtensorMap& tdo, const CUtensorMap& tdq, const BwdArgs& a, const DevCtl& c,
-                            cudaStream_t s);
+                            const CUtensorMap& tdo, const CUtensorMap& tdq, const CUtensorMap& tdk,
+                            const CUtensorMap& tdv, const BwdArgs& a, const DevCtl& c, cudaStream_t s);
+// zero the split accumulators before, and write bf16 dK (x scale), dV from them after, the main kernel
+cudaError_t launch_bwd_kv_zero(const BwdArgs& a, cudaStream_t s);
+cudaError_t launch_bwd_kv_convert(const BwdArgs& a, cudaStream_t s);
+// TMA descriptor for an fp32 [B, N, Hkv, d] dK / dV accumulator: a box of d features x
+// 64 (d = 128) or 128 (d = 64) keys of one (b, head), no swizzle (for TMA reduce-add).
+CUresult make_kv_accum_map(CUtensorMap* map, float* base, int B, int N, int Hkv, int d);
 cudaError_t launch_bwd_main64(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                              const CUtensorMap& tdo, const CUtensorMap& tdq, const BwdArgs& a, const DevCtl& c,
-                              cudaStream_t s);
+                              const CUtensorMap& tdo, const CUtensorMap& tdq, const CUtensorMap& tdk,
+                              const CUtensorMap& tdv, const BwdArgs& a, const DevCtl& c, cudaStream_t s);
 cudaError_t launch_bwd_dq(const BwdArgs& a, cudaStream_t s);
 
 // Chunked-sequence (ring) helpers: merge of partial results, fp32 accumulation, cast.

@@ -154,10 +154,17 @@ int fa_fwd_fp8(const void* Q, const void* K, const void* V, void* O, float* LSE,
  * accumulator [B, N, H, d] plus two fp32 [B, H, roundup(N, 128)] rows
  * (rowsum(dO * O) and LSE * log2 e), each region 256-byte aligned.  This is
  * the O(N) extra memory of the method ("Flash Attention" (karlkratz.de),
- * "Speicherbedarf und Laufzeitverhalten").  Returns 0 for invalid or empty
- * problems.
+ * "Speicherbedarf und Laufzeitverhalten").
+ * For small problems (fewer than three waves of key-tile CTAs on the GPU's 148
+ * SMs) the size also covers two fp32 [B, N, Hkv, d] dK / dV accumulators: with
+ * them the backward splits each key tile's work over several CTAs and sums
+ * their partial dK, dV.  A workspace of only the first three regions is still
+ * accepted (no split).  Returns 0 for invalid or empty problems.
  */
 size_t fa_bwd_workspace_size(int B, int H, int N, int d, int dtype);
+
+/* The same for Hkv K/V heads (fa_bwd_gqa, fa_bwd_window, fa_bwd_blocksparse). */
+size_t fa_bwd_workspace_size_gqa(int B, int H, int Hkv, int N, int d, int dtype);
 
 /*
  * Backward pass by recomputation ("Flash Attention" (karlkratz.de),

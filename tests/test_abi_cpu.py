@@ -94,19 +94,32 @@ def test_backward_validation(L):
 
 
 def test_workspace_is_linear_in_n(L):
-    """The method's extra memory is O(N): the fp32 dQ accumulator plus two rows per (b, h)."""
-    def ws(n):
-        return L.fa_bwd_workspace_size(2, 16, n, 128, 0)
+    """The method's extra memory is O(N): the fp32 dQ accumulator plus two rows per (b, h),
+    and for grids of fewer than three waves of key-tile CTAs, fp32 dK / dV accumulators."""
+    def ws(n, H=16, Hkv=None):
+        return L.fa_bwd_workspace_size_gqa(2, H, H if Hkv is None else Hkv, n, 128, 0)
     B, H, d = 2, 16, 128
-    for n in (128, 4096, 16384):
+    for n in (4096, 16384):  # 1024 / 4096 CTAs: no split
         expect = B * n * H * d * 4 + 2 * B * H * n * 4
         assert ws(n) == expect
+        assert L.fa_bwd_workspace_size(B, H, n, d, 0) == expect
+    # B2 H16 N1024: 256 CTAs but only 8 query tiles per key tile, too few to split;
+    # B1 H4 N4096: 128 CTAs of 32 query tiles, split (causal / windowed walks)
+    assert ws(1024) == B * 1024 * H * d * 4 + 2 * B * H * 1024 * 4
+    assert L.fa_bwd_workspace_size(1, 4, 4096, d, 0) == 4096 * 4 * d * 4 * 3 + 2 * 4 * 4096 * 4
+    # grouped heads shrink the grid: H64 Hkv8 N4096 is 256 CTAs at B1 (split), 1024 at B4 (7 full
+    # waves, no split)
+    assert L.fa_bwd_workspace_size_gqa(1, 64, 8, 4096, 128, 0) == \
+        4096 * 64 * d * 4 + 2 * 64 * 4096 * 4 + 2 * 4096 * 8 * d * 4
+    assert L.fa_bwd_workspace_size_gqa(4, 64, 8, 4096, 128, 0) == 4 * (4096 * 64 * d * 4 + 2 * 64 * 4096 * 4)
     # versus the N x N score matrix standard attention would store (2 bytes each)
     assert ws(16384) < 2 * 16384 * 16384 * H * B
     assert L.fa_bwd_workspace_size(0, 1, 1, 128, 0) == 0
     assert L.fa_bwd_workspace_size(1, 1, 1, 96, 0) == 0
-    # ragged N rounds the per-row arrays up to a multiple of 128
-    assert ws(130) == ((2 * 130 * 16 * 128 * 4 + 255) // 256 * 256) + 2 * ((2 * 16 * 256 * 4 + 255) // 256 * 256)
+    assert L.fa_bwd_workspace_size_gqa(1, 8, 3, 128, 128, 0) == 0
+    # ragged N rounds the per-row arrays up to a multiple of 128 (B4: 2112 CTAs, no split)
+    assert L.fa_bwd_workspace_size(4, 16, 4097, 128, 0) == \
+        ((4 * 4097 * 16 * 128 * 4 + 255) // 256 * 256) + 2 * ((4 * 16 * 4224 * 4 + 255) // 256 * 256)
 
 
 def test_python_binding_refuses_cpu_tensors(L):
