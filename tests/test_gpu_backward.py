@@ -111,8 +111,9 @@ def test_autograd_function_matches_oracle():
 
 @pytest.mark.gpu
 def test_bwd_refuses_what_it_does_not_implement():
+    """The fp32 backward is not implemented: refused, nothing computed."""
     need_gpu()
-    q = torch.zeros(1, 128, 1, 64, dtype=torch.bfloat16, device="cuda")
+    q = torch.zeros(1, 128, 1, 64, dtype=torch.float32, device="cuda")
     lse = torch.zeros(1, 1, 128, device="cuda")
     with pytest.raises(fa.FAError) as e:
         fa.bwd(q, q, q, q, q, lse)
