@@ -20,7 +20,7 @@
 //     mask, take the row max, form P = 2^(S*scale*log2e - m) with the scale
 //     folded into one FFMA, add the row sum, and write P back as bf16;
 //   * lazy rescale: the reference maximum m only moves when a row's maximum
-//     grows by more than 2^8; numerator and denominator share m, so the result
+//     grows by more than 2^12; numerator and denominator share m, so the result
 //     is exact and the O rescale (a TMEM read-modify-write) is rare;
 //   * causal and sliding-window masks: key tiles that no row of the query
 //     tile can see are never loaded or multiplied ("Flash Attention"
@@ -46,7 +46,13 @@ constexpr uint32_t kRegSoftmax = 216;
 constexpr uint32_t kRegOther = 72;
 static_assert(kRegSoftmax >= 168 && kRegOther <= 168, "setmaxnreg direction (launch count 168)");
 static_assert(2 * kRegSoftmax + kRegOther == 3 * 168, "register split must match the launch");
-constexpr float kTau = 8.0f;    // lazy-rescale threshold (log2 units)
+// Lazy-rescale threshold (log2 units).  A stale m leaves every p <= 2^kTau, so
+// l <= 2^kTau * N and |O| <= 2^kTau * N * max|V| stay far inside fp32 for any
+// N < 2^31; bf16 P keeps its relative precision at any scale.  12 rather than
+// 8: inputs with a few large keys (the K-spike workload) otherwise move m on
+// about a fifth of the (query tile, key tile) steps, each a stall of the
+// softmax warps for a read-modify-write of O in TMEM.
+constexpr float kTau = 12.0f;
 // When > 0, one score pair in kPolyEvery takes its exponentials on the FMA pipe
 // (exp2_poly2) instead of the MUFU unit.  Measured on B200 at d = 128 the MUFU
 // is not what limits this kernel (1/4, 1/3 and 1/2 of the pairs on the FMA pipe

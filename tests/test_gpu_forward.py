@@ -107,13 +107,17 @@ def test_bf16_b4_h16_n1024_d64(causal):
 @pytest.mark.gpu
 @pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("causal", [False, True])
-def test_bf16_growing_row_maximum(d, causal):
-    """Scores grow along the keys so the running maximum jumps by far more than
-    the lazy-rescale threshold on many tiles; the oracle handles it exactly."""
+@pytest.mark.parametrize("top", [24.0, 48.0])
+def test_bf16_growing_row_maximum(d, causal, top):
+    """Scores grow along the keys so the running maximum moves by many times the
+    lazy-rescale threshold over a row: with top = 24 by about 8.6 (d = 64) to 12
+    (d = 128) log2 units per key tile, so the kept maximum trails and moves every
+    tile or two; with top = 48 by 17 to 24 per tile, so it moves on every tile.
+    The oracle handles both exactly."""
     need_gpu()
     B, N, H = 1, 1024, 2
     q = torch.full((B, N, H, d), 0.25)
-    ramp = torch.linspace(0.0, 24.0, N).view(1, N, 1, 1)
+    ramp = torch.linspace(0.0, top, N).view(1, N, 1, 1)
     g = torch.Generator().manual_seed(3)
     k = (ramp + 0.05 * torch.randn(B, N, H, d, generator=g)).to(torch.bfloat16)
     v = torch.randn(B, N, H, d, generator=g).to(torch.bfloat16)
