@@ -11,6 +11,13 @@ same generator picks floor(frac * N) sequence positions whose K rows (all
 batches and heads) are multiplied by ``spike`` in float32, which forces large
 jumps of the running row maximum in the online softmax.  The tensors are then
 cast to the working dtype with round-to-nearest-even.
+
+Paged decode inputs (``make_paged_decode``): the same generator draws Q
+[B, H, d], then a page pool K, V [num_pages, page_size, Hkv, d] of standard
+normals, then ``randperm(num_pages)`` which hands out the pool's pages to the
+sequences in order (sequence b takes the next ceil(seqlens[b] / page_size)
+entries), so a sequence's pages are scattered over the pool.  Table entries
+past a sequence's last page are -1.
 """
 
 from __future__ import annotations
@@ -101,3 +108,30 @@ def workload_inputs(w: Workload, *, with_do=None):
     return make_inputs(w.B, w.N, w.H, w.d, seed=w.seed, dtype=w.dtype,
                        spike_frac=w.spike_frac, spike=w.spike,
                        with_do=w.backward if with_do is None else with_do, kv_heads=w.kv_heads)
+
+
+def make_paged_decode(B: int, H: int, Hkv: int, d: int, page_size: int, seqlens, *, seed: int = 0,
+                      spare_pages: int = 0, max_pages: int | None = None):
+    """Return CPU tensors (q, k_cache, v_cache, block_table, seqlens) for one decode step.
+
+    q: [B, H, d] bf16; k_cache, v_cache: [num_pages, page_size, Hkv, d] bf16 with
+    num_pages = the pages the sequences need + ``spare_pages`` (never referenced);
+    block_table: [B, max_pages] int32 (default: the longest sequence's page
+    count), -1 past each sequence's last page; seqlens: [B] int32.
+    """
+    g = torch.Generator(device="cpu").manual_seed(int(seed))
+    lens = [int(x) for x in seqlens]
+    need = [(n + page_size - 1) // page_size for n in lens]
+    num_pages = sum(need) + int(spare_pages)
+    width = max(need + [1]) if max_pages is None else int(max_pages)
+    q = torch.randn((B, H, d), generator=g, dtype=torch.float32)
+    k = torch.randn((num_pages, page_size, Hkv, d), generator=g, dtype=torch.float32)
+    v = torch.randn((num_pages, page_size, Hkv, d), generator=g, dtype=torch.float32)
+    order = torch.randperm(max(num_pages, 1), generator=g)[:num_pages]
+    table = torch.full((B, width), -1, dtype=torch.int32)
+    nxt = 0
+    for b in range(B):
+        table[b, :need[b]] = order[nxt:nxt + need[b]].to(torch.int32)
+        nxt += need[b]
+    return (q.to(torch.bfloat16).contiguous(), k.to(torch.bfloat16).contiguous(), v.to(torch.bfloat16).contiguous(),
+            table, torch.tensor(lens, dtype=torch.int32))

@@ -9,11 +9,13 @@ from .attention import (  # noqa: F401
     backward,
     backward_head,
     blocked_forward_head,
+    decode_paged,
     forward,
     forward_head,
     forward_rows_head,
     hidden_keys,
     kv_head,
+    paged_rows,
     probs_head,
     scores_head,
 )

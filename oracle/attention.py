@@ -57,6 +57,15 @@ Readings where the pages are silent (all recorded in the design notes):
   score matrix (one per query head, or one shared); a row whose blocks are all
   0 sees no key and gets O = 0, LSE = -inf.
 
+* a paged KV cache ("Flash Attention" (Ultralytics glossary), "Flash Attention
+  и смежные понятия", PagedAttention: the cache lives in fixed-size pages and
+  the attention kernel reads keys and values from them) is a pool
+  [num_pages, page_size, Hkv, d] plus a per-sequence page list: position j of
+  sequence b is slot j % page_size of page block_table[b, j // page_size].  A
+  decode step is one query per sequence attending to all seqlens[b] cached
+  positions (none hidden); a sequence with no cached position gets O = 0,
+  LSE = -inf.
+
 ``blocked_forward_head`` restates the pages' online-softmax algorithm (key
 blocks streamed, running row max and sum, rescale when the max grows) and is
 used only to pin the oracle: blocked and full results must agree.
@@ -80,6 +89,8 @@ __all__ = [
     "forward",
     "backward",
     "kv_head",
+    "paged_rows",
+    "decode_paged",
 ]
 
 
@@ -344,3 +355,54 @@ def _to_numpy(t):
             t = t.float()
         return t.cpu().numpy()
     return np.asarray(t)
+
+
+def paged_rows(cache, table_row, length: int) -> np.ndarray:
+    """The first ``length`` cached rows of one sequence, gathered from a page pool.
+
+    cache: [num_pages, page_size, ...] (numpy or CPU torch); table_row: the
+    sequence's page list.  Position j sits in slot j % page_size of page
+    table_row[j // page_size] ("Flash Attention" (Ultralytics glossary), "Flash
+    Attention и смежные понятия", PagedAttention: keys and values are read from
+    fixed-size pages).  Returns [length, ...] float64.
+    """
+    cache = _f64(_to_numpy(cache))
+    table_row = np.asarray(_to_numpy(table_row), dtype=np.int64)
+    page_size = cache.shape[1]
+    out = np.empty((length,) + cache.shape[2:])
+    for j in range(length):
+        out[j] = cache[table_row[j // page_size], j % page_size]
+    return out
+
+
+def decode_paged(Q, K_cache, V_cache, block_table, seqlens, scale: float):
+    """One decode step of attention over a paged KV cache.
+
+    Q: [B, H, d] (one new query per sequence); K_cache, V_cache:
+    [num_pages, page_size, Hkv, d]; block_table: [B, max_pages] page indices;
+    seqlens: [B] cached positions per sequence.  Query head h of sequence b
+    attends, with K/V head ``kv_head(h)``, to the seqlens[b] rows that
+    ``paged_rows`` gathers: the plain definition (``forward_rows_head``, no
+    mask) on the gathered rows.  Returns O [B, H, d] and LSE [B, H] (float64);
+    a sequence with no cached position gets O = 0 and LSE = -inf.
+    """
+    Q = _f64(_to_numpy(Q))
+    K_cache, V_cache = (_f64(_to_numpy(t)) for t in (K_cache, V_cache))
+    table = np.asarray(_to_numpy(block_table), dtype=np.int64)
+    lens = np.asarray(_to_numpy(seqlens), dtype=np.int64)
+    nb, nh, d = Q.shape
+    hkv = K_cache.shape[2]
+    O = np.zeros((nb, nh, V_cache.shape[3]))
+    LSE = np.full((nb, nh), -np.inf)
+    for b in range(nb):
+        n = int(lens[b])
+        if n == 0:
+            continue
+        k_rows = paged_rows(K_cache, table[b], n)  # [n, Hkv, d]
+        v_rows = paged_rows(V_cache, table[b], n)
+        for h in range(nh):
+            g = kv_head(h, nh, hkv)
+            o, lse = forward_rows_head(Q[b, h][None, :], k_rows[:, g], v_rows[:, g], [0], scale, False)
+            O[b, h] = o[0]
+            LSE[b, h] = lse[0]
+    return O, LSE

@@ -705,3 +705,128 @@ def test_blocksparse_mutants_are_caught():
         return A.forward_head(q, k, v, scale, causal, window, None)
     assert _caught(pin_blocksparse_rowwise, dense)
 
+
+
+# ---------------------------------------------------------------------------
+# Paged KV cache, one decode step ("Flash Attention" (Ultralytics glossary),
+# "Flash Attention и смежные понятия", PagedAttention)
+# ---------------------------------------------------------------------------
+
+def _paged_case(seed, lens, H=6, Hkv=2, d=5, P=4, spare=3):
+    """Contiguous per-sequence K/V, and a pool holding them in shuffled pages.
+
+    The pool is built here by slicing each sequence into page-sized chunks and
+    storing chunk c of sequence b at page perm[first page of b + c]; every pool
+    row that holds no cached position is NaN, so reading one poisons the result.
+    """
+    rng = np.random.default_rng(seed)
+    B = len(lens)
+    q = rng.standard_normal((B, H, d))
+    ks = [rng.standard_normal((n, Hkv, d)) for n in lens]
+    vs = [rng.standard_normal((n, Hkv, d)) for n in lens]
+    npages = [-(-n // P) for n in lens]
+    total = sum(npages) + spare
+    perm = rng.permutation(total)
+    kc = np.full((total, P, Hkv, d), np.nan)
+    vc = np.full((total, P, Hkv, d), np.nan)
+    table = np.full((B, max(npages + [1]) + 1), -7, dtype=np.int64)
+    first = 0
+    for b, n in enumerate(lens):
+        for c in range(npages[b]):
+            page = perm[first + c]
+            table[b, c] = page
+            rows = slice(c * P, min(n, (c + 1) * P))
+            kc[page, : rows.stop - rows.start] = ks[b][rows]
+            vc[page, : rows.stop - rows.start] = vs[b][rows]
+        first += npages[b]
+    return q, ks, vs, kc, vc, table, np.asarray(lens)
+
+
+def pin_paged_sdpa(decode=A.decode_paged):
+    """One decode step against torch SDPA (fp64, CPU, enable_gqa) on each sequence's contiguous K/V."""
+    worst = 0.0
+    for seed, lens, H, Hkv, P in ((1, [7, 1, 12, 4], 6, 2, 4), (2, [9, 16, 3], 4, 4, 8), (3, [5, 11], 6, 1, 3)):
+        q, ks, vs, kc, vc, table, lens_a = _paged_case(seed, lens, H=H, Hkv=Hkv, P=P)
+        o, lse = decode(q, kc, vc, table, lens_a, 0.7)
+        for b, n in enumerate(lens):
+            tq = torch.tensor(q[b][:, None, :])            # [H, 1, d]
+            tk = torch.tensor(ks[b].transpose(1, 0, 2))     # [Hkv, n, d]
+            tv = torch.tensor(vs[b].transpose(1, 0, 2))
+            ref = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, scale=0.7, enable_gqa=True)
+            s = 0.7 * torch.einsum("hd,hnd->hn", tq[:, 0], tk.repeat_interleave(H // Hkv, 0))
+            ref_lse = torch.logsumexp(s, dim=1)
+            err = max(float(np.max(np.abs(o[b] - ref[:, 0].numpy()))), float(np.max(np.abs(lse[b] - ref_lse.numpy()))))
+            worst = max(worst, err if np.isfinite(err) else math.inf)
+    return worst
+
+
+def pin_paged_special_cases(decode=A.decode_paged):
+    """Closed forms: one cached position gives O = v_0, LSE = scale <q, k_0>; none gives O = 0, LSE = -inf."""
+    q, ks, vs, kc, vc, table, lens = _paged_case(4, [1, 0, 1], H=4, Hkv=2, P=4)
+    o, lse = decode(q, kc, vc, table, lens, 0.9)
+    worst = 0.0
+    for b in (0, 2):
+        for h in range(4):
+            g = h // 2
+            worst = max(worst, float(np.max(np.abs(o[b, h] - vs[b][0, g]))),
+                        abs(float(lse[b, h]) - 0.9 * float(q[b, h] @ ks[b][0, g])))
+    ok_empty = np.all(o[1] == 0.0) and np.all(np.isneginf(lse[1]))
+    return worst if ok_empty and np.isfinite(worst) else math.inf
+
+
+def test_paged_decode_matches_sdpa_on_contiguous_rows():
+    assert pin_paged_sdpa() < 1e-12
+
+
+def test_paged_decode_special_cases():
+    assert pin_paged_special_cases() < 1e-12
+
+
+def test_paged_decode_with_an_identity_table_is_the_plain_forward():
+    """Pages laid out in order reduce the gather to slicing the flattened pool."""
+    rng = np.random.default_rng(9)
+    P, n, Hkv, H, d = 4, 10, 2, 4, 3
+    kc = rng.standard_normal((3, P, Hkv, d))
+    vc = rng.standard_normal((3, P, Hkv, d))
+    q = rng.standard_normal((1, H, d))
+    o, lse = A.decode_paged(q, kc, vc, np.arange(3)[None, :], np.array([n]), 0.4)
+    kf, vf = kc.reshape(-1, Hkv, d)[:n], vc.reshape(-1, Hkv, d)[:n]
+    for h in range(H):
+        oh, lh = A.forward_head(q[0, h][None, :], kf[:, h // 2], vf[:, h // 2], 0.4, False)
+        assert np.allclose(o[0, h], oh[0], rtol=0, atol=1e-14) and abs(lse[0, h] - lh[0]) < 1e-14
+
+
+def _mut_paged(kind):
+    def decode(Q, Kc, Vc, table, lens, scale):
+        nb, nh, _ = Q.shape
+        hkv, P = Kc.shape[2], Kc.shape[1]
+        O = np.zeros(Q.shape)
+        LSE = np.full((nb, nh), -np.inf)
+        for b in range(nb):
+            n = int(lens[b]) + (1 if kind == "one_row_too_many" else 0)
+            if n == 0:
+                continue
+            row = table[(b + 1) % nb] if kind == "wrong_sequence" else table[b]
+            if kind == "page_slot_swapped":
+                idx = [(row[j % P], j // P) for j in range(n)]
+            else:
+                idx = [(row[j // P], j % P) for j in range(n)]
+            kr = np.stack([Kc[p, s] for p, s in idx])
+            vr = np.stack([Vc[p, s] for p, s in idx])
+            for h in range(nh):
+                g = h % hkv if kind == "interleaved_heads" else A.kv_head(h, nh, hkv)
+                o, l = A.forward_rows_head(Q[b, h][None, :], kr[:, g], vr[:, g], [0], scale, False)
+                O[b, h], LSE[b, h] = o[0], l[0]
+        return O, LSE
+    return decode
+
+
+@pytest.mark.parametrize("kind", ["page_slot_swapped", "one_row_too_many", "wrong_sequence", "interleaved_heads"])
+def test_paged_decode_mutants_are_caught(kind):
+    with np.errstate(invalid="ignore", over="ignore"):
+        try:
+            worst = pin_paged_sdpa(decode=_mut_paged(kind))
+        except (IndexError, ValueError):
+            worst = math.inf  # the mistake reads outside the pool or table
+    assert worst > 1e-6
+    assert pin_paged_sdpa(decode=_mut_paged("none")) < 1e-12
