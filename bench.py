@@ -44,6 +44,8 @@ sys.path.insert(0, str(ROOT))
 
 METRIC = "attention TFLOP/s (fwd, fwd+bwd) bf16 on 1 B200 and % of dense BF16 tensor peak"
 WORKLOAD = dict(B=1, H=32, N=16384, d=128, causal=False, spike_frac=0.01, spike=3.0)
+DECODE_WORKLOAD = dict(B=64, H=64, Hkv=8, d=128, page=16, lo=512, hi=8192, seed=21)
+DECODE_NAME = "bf16 paged decode B64 H64 Hkv8 d128, 16-token pages, lengths 512..8192"
 WORKLOAD_NAME = "bf16 fwd+bwd B1 H32 N16384 d128 non-causal, K rows x3 at 1% of positions"
 FALLBACK_PEAK_TFLOPS = 1590.0  # earlier burst measurement of cuBLAS bf16 on this machine
 
@@ -59,6 +61,13 @@ def read_peaks():
         j = json.loads(p.read_text())
         return float(j["bf16_tflops"]), float(j.get("bf16_tflops_sustained", j["bf16_tflops"])), "measured"
     return FALLBACK_PEAK_TFLOPS, 1400.0, "fallback"
+
+
+def read_hbm_peak():
+    p = ROOT / "MEASURED_PEAKS.json"
+    if p.exists():
+        return float(json.loads(p.read_text())["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
 
 
 def read_profile_traffic(kernel_key: str):
@@ -403,6 +412,42 @@ def run_ours(args, world, rank, local):
                "inputs": "Q, K, V of the same workload as e4m3 codes with per-tensor scales"}
         del codes, o8
 
+    # ---- one decode step over a paged KV cache (HBM-bound; its own workload) ----
+    # 64 sequences, 64 query heads on 8 K/V heads, d 128, 16-token pages handed
+    # out in shuffled order, lengths uniform in [512, 8192]: 1.16 GB of K/V per
+    # step, larger than L2.
+    dw = DECODE_WORKLOAD
+    dlens = I.decode_lengths(dw["B"], dw["lo"], dw["hi"], seed=dw["seed"] + rank)
+    dq_, dk_, dv_, dt_, ds_ = (t.to(dev) for t in I.make_paged_decode(
+        dw["B"], dw["H"], dw["Hkv"], dw["d"], dw["page"], dlens, seed=dw["seed"] + rank))
+    dws = torch.empty(max(1, fa.decode_workspace_size(dw["B"], dw["H"], dw["Hkv"], dw["d"], dw["page"],
+                                                      dt_.shape[1])), dtype=torch.uint8, device=dev)
+    d_o, d_l = fa.decode_paged(dq_, dk_, dv_, dt_, ds_, workspace=dws)
+    for _ in range(5):
+        fa.decode_paged(dq_, dk_, dv_, dt_, ds_, out=d_o, lse=d_l, workspace=dws)
+    nd = max(5, min(4 * args.steps, 50))
+    ed0, ed1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    ed0.record(stream)
+    for _ in range(nd):
+        fa.decode_paged(dq_, dk_, dv_, dt_, ds_, out=d_o, lse=d_l, workspace=dws)
+    ed1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    rc, detail = fa.last_device_status()
+    if rc != 0:
+        raise RuntimeError(f"device status {rc} ({detail:#x}) after the decode steps")
+    d_ms = slowest(ed0.elapsed_time(ed1)) / nd
+    d_bytes = (sum(dlens) * dw["Hkv"] * dw["d"] * 2 * 2 + 2 * dw["B"] * dw["H"] * dw["d"] * 2
+               + dw["B"] * dw["H"] * 4 + dw["B"] * (dt_.shape[1] + 1) * 4)
+    hbm, hbm_src = read_hbm_peak()
+    decode = {"workload": DECODE_NAME, "gbs": d_bytes / (d_ms * 1e-3) / 1e9, "us": d_ms * 1e3, "launches": nd,
+              "bytes_per_launch": d_bytes, "bound": "hbm", "peak_gbs": hbm, "peak_source": f"{hbm_src} copy",
+              "frac_of_peak": d_bytes / (d_ms * 1e-3) / 1e9 / hbm,
+              "bytes": "K and V rows of every cached position once, Q and O, LSE, block table and lengths"}
+    del dq_, dk_, dv_, dt_, ds_, dws, d_o, d_l
+
     # ---- end to end through the public API with host buffers ----
     # Every step copies its four inputs from pinned host memory and its five
     # outputs back.  Two device buffer sets and two copy streams pipeline the
@@ -486,6 +531,7 @@ def run_ours(args, world, rank, local):
         "peak_tflops": {"burst": peak_burst, "sustained": peak_sustained, "used": peak, "source": peak_src},
         "roofline": roofline,
         "fwd_fp8": fp8,
+        "decode_paged": decode,
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "steps": e_steps, "ms_per_step": e2e_ms / e_steps,
                 "how": "pinned host -> device inputs and device -> pinned host outputs every step, "
@@ -531,6 +577,25 @@ def run_profile_case(args):
     print(json.dumps({"profile_case": w, "ok": True}))
 
 
+def run_profile_decode():
+    """Small case for ncu section captures of the paged decode: 2 launches on 32
+    sequences (lengths 512..8192, 64 query heads on 8 K/V heads, d 128, 16-token
+    pages): about 0.6 GB of K/V, more than the L2, well under the device memory."""
+    import torch
+
+    import exact_io_aware_51_b200 as fa
+    from exact_io_aware_51_b200 import inputs as I
+    lens = I.decode_lengths(32, 512, 8192, seed=21)
+    q, k, v, t, s = (x.cuda() for x in I.make_paged_decode(32, 64, 8, 128, 16, lens, seed=21))
+    for _ in range(2):
+        fa.decode_paged(q, k, v, t, s)
+    torch.cuda.synchronize()
+    rc, detail = fa.last_device_status()
+    if rc != 0:
+        raise RuntimeError(f"device status {rc} ({detail:#x})")
+    print(json.dumps({"profile_case": "decode B32 H64 Hkv8 d128 P16", "ok": True}))
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -541,7 +606,12 @@ def main():
     ap.add_argument("--profile-case", action="store_true",
                     help="run only the small profiling case (2 x fwd + bwd, B1 H64 N4096 d128) for ncu")
     ap.add_argument("--profile-causal", action="store_true", help="with --profile-case: also the causal pair")
+    ap.add_argument("--profile-decode", action="store_true",
+                    help="run only the small paged-decode profiling case (2 launches, B32) for ncu")
     args = ap.parse_args()
+    if args.profile_decode:
+        run_profile_decode()
+        return
     if args.profile_case:
         run_profile_case(args)
         return

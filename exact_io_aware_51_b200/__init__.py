@@ -20,7 +20,7 @@ import torch
 
 __all__ = [
     "FAError", "FA_BF16", "FA_FP32", "lib", "lib_path", "fwd", "fwd_fp8", "bwd", "bwd_workspace_size",
-    "merge_partial", "accumulate", "cast_bf16",
+    "merge_partial", "accumulate", "cast_bf16", "decode_paged", "decode_workspace_size",
     "last_device_status", "set_wait_limit_ms", "debug_inject", "debug_umma", "debug_umma_f8", "status_string",
     "set_kernel_events",
     "attention", "EXPORTED",
@@ -37,7 +37,7 @@ EXPORTED = ("fa_fwd", "fa_bwd_workspace_size", "fa_bwd", "fa_status_string", "fa
             "fa_version", "fa_set_kernel_events", "fa_bwd_static_scratch", "fa_fwd_gqa", "fa_bwd_gqa",
             "fa_fwd_window", "fa_bwd_window", "fa_debug_umma_f8", "fa_fwd_fp8",
             "fa_fwd_blocksparse", "fa_bwd_blocksparse", "fa_merge_partial", "fa_accumulate_bf16",
-            "fa_cast_bf16", "fa_bwd_workspace_size_gqa")
+            "fa_cast_bf16", "fa_bwd_workspace_size_gqa", "fa_decode_paged", "fa_decode_workspace_size")
 
 
 class FAError(RuntimeError):
@@ -93,6 +93,10 @@ def lib() -> ctypes.CDLL:
     L.fa_fwd_window.restype = i
     L.fa_bwd_window.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, i, vp, sz, vp]
     L.fa_bwd_window.restype = i
+    L.fa_decode_paged.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, f, vp, sz, vp]
+    L.fa_decode_paged.restype = i
+    L.fa_decode_workspace_size.argtypes = [i, i, i, i, i, i]
+    L.fa_decode_workspace_size.restype = sz
     L.fa_status_string.argtypes = [i]
     L.fa_status_string.restype = ctypes.c_char_p
     L.fa_last_cuda_error.argtypes = []
@@ -234,6 +238,56 @@ def fwd_fp8(q, k, v, scale_q: float, scale_k: float, scale_v: float, causal: boo
                           _stream_handle(stream, q.device))
     if rc != 0:
         raise FAError(rc, "fa_fwd_fp8")
+    return o, l
+
+
+def decode_workspace_size(B: int, H: int, Hkv: int, d: int, page_size: int, max_pages: int) -> int:
+    """Workspace bytes with which ``decode_paged`` splits long sequences as it would unconstrained."""
+    return int(lib().fa_decode_workspace_size(B, H, Hkv, d, page_size, max_pages))
+
+
+def decode_paged(q, k_cache, v_cache, block_table, seqlens, scale: float | None = None, out=None, lse=None,
+                 workspace=None, stream=None):
+    """One decode step over a paged KV cache (fa_decode_paged): returns (o [B, H, d] bf16, lse [B, H] fp32).
+
+    q: [B, H, d] bf16; k_cache, v_cache: [num_pages, page_size, Hkv, d] bf16;
+    block_table: [B, max_pages] int32; seqlens: [B] int32; all on one CUDA
+    device.  ``workspace`` (uint8 cuda tensor) defaults to a fresh buffer of
+    ``decode_workspace_size`` bytes; pass one to avoid the allocation.
+    """
+    if q.dim() != 3 or k_cache.dim() != 4:
+        raise ValueError("expected q [B, H, d] and k_cache, v_cache [num_pages, page_size, Hkv, d]")
+    B, H, d = q.shape
+    num_pages, page_size, Hkv, dk = k_cache.shape
+    if v_cache.shape != k_cache.shape or dk != d:
+        raise ValueError("k_cache and v_cache must be [num_pages, page_size, Hkv, d] with q's d")
+    if block_table.dim() != 2 or block_table.shape[0] != B or seqlens.shape != (B,):
+        raise ValueError("block_table must be [B, max_pages] and seqlens [B]")
+    for t in (q, k_cache, v_cache):
+        if t.dtype != torch.bfloat16:
+            raise TypeError("decode_paged takes bfloat16 q, k_cache, v_cache")
+    for t in (block_table, seqlens):
+        if t.dtype != torch.int32:
+            raise TypeError("block_table and seqlens must be int32")
+    for t in (q, k_cache, v_cache, block_table, seqlens):
+        if not t.is_contiguous():
+            raise ValueError("decode_paged tensors must be contiguous")
+        if t.device != q.device:
+            raise ValueError("decode_paged tensors must share one device")
+    if not q.is_cuda:
+        raise ValueError("tensors must live on a CUDA device (there is no CPU path)")
+    max_pages = block_table.shape[1]
+    o = torch.empty((B, H, d), dtype=torch.bfloat16, device=q.device) if out is None else out
+    l = torch.empty((B, H), dtype=torch.float32, device=q.device) if lse is None else lse
+    if workspace is None:
+        n = decode_workspace_size(B, H, Hkv, d, page_size, max(max_pages, 1))
+        workspace = torch.empty(max(n, 1), dtype=torch.uint8, device=q.device)
+    rc = lib().fa_decode_paged(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), block_table.data_ptr(),
+                               seqlens.data_ptr(), o.data_ptr(), l.data_ptr(), B, H, Hkv, d, page_size, num_pages,
+                               max_pages, _scale(scale, d), workspace.data_ptr(), workspace.numel(),
+                               _stream_handle(stream, q.device))
+    if rc != 0:
+        raise FAError(rc, "fa_decode_paged")
     return o, l
 
 

@@ -23,7 +23,7 @@ BUILD = PKG / "_build"
 LIB = PKG / "libfa.so"
 SOURCES = ("fa_api.cu", "fa_fwd_bf16.cu", "fa_fwd_fp8.cu", "fa_fwd_f32.cu", "fa_bwd.cu", "fa_probe.cu",
            "fa_bwd_static.cu", "fa_ring.cu",
-           "fa_bwd64.cu")
+           "fa_bwd64.cu", "fa_decode.cu")
 ARCH = ("-gencode", "arch=compute_100a,code=sm_100a")
 FLAGS = ("-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall",
          "--expt-relaxed-constexpr")

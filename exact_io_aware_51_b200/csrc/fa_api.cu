@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstdint>
@@ -229,6 +230,19 @@ CUresult make_tile_map(CUtensorMap* map, const void* base, int B, int N, int H, 
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
 }
 
+CUresult make_paged_map(CUtensorMap* map, const void* base, int num_pages, int page_size, int Hkv, int d) {
+  if (!encoder()) return CUDA_ERROR_NOT_FOUND;
+  // dims innermost first: (K/V head, feature), pool row = page * page_size + slot
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(Hkv) * d,
+                              static_cast<cuuint64_t>(num_pages) * static_cast<cuuint64_t>(page_size)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(Hkv) * d * 2};
+  const cuuint32_t box[2] = {64u, static_cast<cuuint32_t>(page_size < 64 ? page_size : 64)};
+  const cuuint32_t estr[2] = {1u, 1u};
+  return g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+}
+
 CUresult make_tile_map_e4m3(CUtensorMap* map, const void* base, int B, int N, int H, int d, int rows) {
   if (!encoder()) return CUDA_ERROR_NOT_FOUND;
   const cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(H),
@@ -306,6 +320,7 @@ const char* fa_status_string(int status) {
     case FA_ERR_LAUNCH: return "CUDA call failed (see fa_last_cuda_error)";
     case FA_ERR_DEVICE_TIMEOUT: return "a kernel wait exceeded its limit; outputs of that launch are undefined";
     case FA_ERR_TOO_LARGE: return "problem exceeds a size limit";
+    case FA_ERR_DEVICE_INPUT: return "device-side input out of range (sequence length or page index)";
     default: return "unknown status";
   }
 }
@@ -336,6 +351,7 @@ int fa_last_device_status(void* stream, int* detail) {
   e = cudaMemcpy(st->status, &zero, sizeof(int), cudaMemcpyHostToDevice);
   if (e != cudaSuccess) return fail_cuda(e);
   if (detail) *detail = v;
+  if (v & kDevBadInput) return FA_ERR_DEVICE_INPUT;
   return v ? FA_ERR_DEVICE_TIMEOUT : FA_OK;
 }
 
@@ -675,6 +691,120 @@ int fa_debug_umma_f8(const void* A, const void* B, float* D, int N, int b_mn_maj
   if (rc) return rc;
   cudaError_t e =
       launch_umma_probe_f8(A, B, D, N, b_mn_major ? 1 : 0, a_tmem ? 1 : 0, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail_cuda(e);
+  return FA_OK;
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// One decode step over a paged KV cache
+// ---------------------------------------------------------------------------
+namespace {
+
+struct DecodePlan {
+  int hgroups, splits, chunk;
+  size_t ws;  // workspace bytes the plan needs (0 with one chunk)
+};
+
+bool pow2_in(int x, int lo, int hi) { return x >= lo && x <= hi && (x & (x - 1)) == 0; }
+
+int check_decode(int B, int H, int Hkv, int d, int page_size, int num_pages, int max_pages, float scale) {
+  if (B < 0 || H < 1 || num_pages < 1 || max_pages < 1) return FA_ERR_INVALID_ARG;
+  int rc = check_kv_heads(H, Hkv);
+  if (rc) return rc;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (!pow2_in(page_size, 8, 4096)) return FA_ERR_UNSUPPORTED;
+  if ((rc = check_scale(scale))) return rc;
+  const long long hg = (H / Hkv + 15) / 16;
+  if (static_cast<long long>(num_pages) * page_size > 0x7fffffffLL ||
+      static_cast<long long>(max_pages) * page_size > 0x7fffffffLL || B > 65535 || Hkv * hg > 65535)
+    return FA_ERR_TOO_LARGE;
+  return FA_OK;
+}
+
+size_t decode_ws_bytes(int B, int H, int d, int splits) {
+  if (splits <= 1) return 0;
+  const size_t rows = static_cast<size_t>(splits) * B * H;
+  return align256(rows * d * sizeof(float)) + align256(rows * sizeof(float));
+}
+
+// Chunks per (sequence, head group): enough CTAs for two waves at two CTAs per SM,
+// at least four 64-key tiles per chunk, and no more than the workspace holds.
+DecodePlan decode_plan(int B, int H, int Hkv, int d, int page_size, int max_pages, size_t ws_cap) {
+  DecodePlan p;
+  p.hgroups = (H / Hkv + 15) / 16;
+  const long long max_keys = static_cast<long long>(max_pages) * page_size;
+  const long long tiles = (max_keys + 63) / 64;
+  const long long ctas = static_cast<long long>(B) * Hkv * p.hgroups;
+  long long want = ctas > 0 ? (4 * 148 + ctas - 1) / ctas : 1;
+  want = std::max(1LL, std::min(want, tiles / 4));
+  for (;;) {
+    const long long chunk_tiles = (tiles + want - 1) / want;
+    p.splits = static_cast<int>((tiles + chunk_tiles - 1) / chunk_tiles);
+    p.chunk = static_cast<int>(chunk_tiles * 64);
+    p.ws = decode_ws_bytes(B, H, d, p.splits);
+    if (p.splits == 1 || p.ws <= ws_cap) break;
+    want = p.splits - 1;
+  }
+  return p;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t fa_decode_workspace_size(int B, int H, int Hkv, int d, int page_size, int max_pages) {
+  if (check_decode(B, H, Hkv, d, page_size, 1, max_pages, 1.0f) != FA_OK) return 0;
+  return decode_plan(B, H, Hkv, d, page_size, max_pages, SIZE_MAX).ws;
+}
+
+int fa_decode_paged(const void* Q, const void* K_cache, const void* V_cache, const int* block_table,
+                    const int* seqlens, void* O, float* LSE, int B, int H, int Hkv, int d, int page_size,
+                    int num_pages, int max_pages, float scale, void* workspace, size_t workspace_bytes,
+                    void* stream) {
+  int rc = check_decode(B, H, Hkv, d, page_size, num_pages, max_pages, scale);
+  if (rc) return rc;
+  if (B == 0) return FA_OK;
+  if (!Q || !K_cache || !V_cache || !block_table || !seqlens || !O || !LSE) return FA_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K_cache) || !aligned16(V_cache) || !aligned16(O) ||
+      (reinterpret_cast<uintptr_t>(LSE) & 3u) || (reinterpret_cast<uintptr_t>(block_table) & 3u) ||
+      (reinterpret_cast<uintptr_t>(seqlens) & 3u))
+    return FA_ERR_MISALIGNED;
+  if (workspace && !aligned16(workspace)) return FA_ERR_WORKSPACE;
+  DeviceState* st = nullptr;
+  if ((rc = device_state(&st))) return rc;
+  const DecodePlan plan = decode_plan(B, H, Hkv, d, page_size, max_pages, workspace ? workspace_bytes : 0);
+  DecodeArgs a;
+  a.B = B;
+  a.H = H;
+  a.Hkv = Hkv;
+  a.d = d;
+  a.page_size = page_size;
+  a.num_pages = num_pages;
+  a.max_pages = max_pages;
+  a.hgroups = plan.hgroups;
+  a.splits = plan.splits;
+  a.chunk = plan.chunk;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.Q = Q;
+  a.block_table = block_table;
+  a.seqlens = seqlens;
+  a.O = O;
+  a.LSE = LSE;
+  const size_t rows = static_cast<size_t>(plan.splits) * B * H;
+  a.Opart = plan.splits > 1 ? static_cast<float*>(workspace) : nullptr;
+  a.LSEpart = plan.splits > 1 ? reinterpret_cast<float*>(static_cast<char*>(workspace) + align256(rows * d * 4))
+                              : nullptr;
+  CUtensorMap tk, tv;
+  CUresult r;
+  if ((r = make_paged_map(&tk, K_cache, num_pages, page_size, Hkv, d)) != CUDA_SUCCESS ||
+      (r = make_paged_map(&tv, V_cache, num_pages, page_size, Hkv, d)) != CUDA_SUCCESS)
+    return fail_encode(r);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (t_ev_start) cudaEventRecord(t_ev_start, s);
+  cudaError_t e = launch_decode(tk, tv, a, make_ctl(*st), s);
+  if (t_ev_stop && e == cudaSuccess) cudaEventRecord(t_ev_stop, s);
   if (e != cudaSuccess) return fail_cuda(e);
   return FA_OK;
 }

@@ -87,6 +87,36 @@ CUresult make_dq_accum_map(CUtensorMap* map, float* base, int B, int N, int H, i
 // a box of 32 features x 128 sequence positions of one (b, h), 128-byte swizzle.
 CUresult make_dq_accum_map_sw128(CUtensorMap* map, float* base, int B, int N, int H, int d);
 
+// Status-word bit a kernel sets when device-side input data (a sequence length
+// or a page index) is out of range; the low bits name the check.
+constexpr int kDevBadInput = 0x2000;
+
+// One decode step over a paged KV cache: Q [B, H, d] (one query per sequence),
+// K, V pools [num_pages, page_size, Hkv, d], block_table [B, max_pages],
+// seqlens [B]; both int32 arrays live on the device.
+struct DecodeArgs {
+  int B, H, Hkv, d;
+  int page_size, num_pages, max_pages;
+  int hgroups;       // CTAs per K/V head: ceil((H / Hkv) / 16) groups of <= 16 query heads
+  int splits;        // key chunks per (sequence, head group)
+  int chunk;         // keys per chunk (a multiple of 64)
+  float scale_log2;  // softmax scale * log2(e)
+  const void* Q;
+  const int* block_table;
+  const int* seqlens;
+  void* O;           // [B, H, d] bf16
+  float* LSE;        // [B, H] natural log
+  float* Opart;      // splits > 1: [splits, B, H, d] fp32, normalised per chunk
+  float* LSEpart;    // splits > 1: [splits, B, H] natural log (-inf: no key in the chunk)
+};
+
+// TMA descriptor for a paged K or V pool [num_pages, page_size, Hkv, d] bf16 viewed
+// as [num_pages * page_size rows][Hkv * d]: a box of min(page_size, 64) rows x 64
+// features, 128-byte swizzle.
+CUresult make_paged_map(CUtensorMap* map, const void* base, int num_pages, int page_size, int Hkv, int d);
+cudaError_t launch_decode(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeArgs& a, const DevCtl& c,
+                          cudaStream_t s);
+
 // Kernel launchers (each returns the cudaError_t of the launch).
 cudaError_t launch_fwd_bf16(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const FwdArgs& a, const DevCtl& c, cudaStream_t s);

@@ -17,7 +17,8 @@ Paged decode inputs (``make_paged_decode``): the same generator draws Q
 normals, then ``randperm(num_pages)`` which hands out the pool's pages to the
 sequences in order (sequence b takes the next ceil(seqlens[b] / page_size)
 entries), so a sequence's pages are scattered over the pool.  Table entries
-past a sequence's last page are -1.
+past a sequence's last page are -1.  ``decode_lengths`` draws a batch's
+sequence lengths uniformly from [lo, hi] with its own seeded generator.
 """
 
 from __future__ import annotations
@@ -135,3 +136,9 @@ def make_paged_decode(B: int, H: int, Hkv: int, d: int, page_size: int, seqlens,
         nxt += need[b]
     return (q.to(torch.bfloat16).contiguous(), k.to(torch.bfloat16).contiguous(), v.to(torch.bfloat16).contiguous(),
             table, torch.tensor(lens, dtype=torch.int32))
+
+
+def decode_lengths(B: int, lo: int, hi: int, *, seed: int = 0) -> list:
+    """B sequence lengths drawn uniformly from [lo, hi] (a seeded CPU generator)."""
+    g = torch.Generator(device="cpu").manual_seed(int(seed))
+    return [int(x) for x in torch.randint(lo, hi + 1, (B,), generator=g)]

@@ -63,7 +63,8 @@ enum {
   FA_ERR_ARCH = -5,            /* current device is not compute capability 10.0 */
   FA_ERR_LAUNCH = -6,          /* a CUDA call failed; see fa_last_cuda_error() */
   FA_ERR_DEVICE_TIMEOUT = -7,  /* a kernel's bounded wait expired (see fa_last_device_status) */
-  FA_ERR_TOO_LARGE = -8        /* a size limit above is exceeded */
+  FA_ERR_TOO_LARGE = -8,       /* a size limit above is exceeded */
+  FA_ERR_DEVICE_INPUT = -9     /* a kernel found device-side input out of range (see fa_last_device_status) */
 };
 
 /*
@@ -276,6 +277,50 @@ int fa_accumulate_bf16(float* acc, const void* part, long long n, int init, void
 /* out[i] = bf16(in[i]) (round to nearest even) for i < n; n a multiple of 8. */
 int fa_cast_bf16(void* out, const float* in, long long n, void* stream);
 
+/*
+ * One decode step of attention over a paged KV cache ("Flash Attention"
+ * (Ultralytics glossary), "Flash Attention и смежные понятия", PagedAttention:
+ * the KV cache is kept in fixed-size pages and the attention kernel reads keys
+ * and values from those pages).
+ *   Q            [B, H, d] bf16: the one new query of each sequence.
+ *   K_cache,     [num_pages, page_size, Hkv, d] bf16 page pools; position j of
+ *   V_cache      sequence b is slot j % page_size of page
+ *                block_table[b * max_pages + j / page_size].
+ *   block_table  [B, max_pages] int32 device array of page indices; only the
+ *                first ceil(seqlens[b] / page_size) entries of a row are read.
+ *   seqlens      [B] int32 device array: cached positions of each sequence,
+ *                0 <= seqlens[b] <= max_pages * page_size.
+ *   O            [B, H, d] bf16 output;  LSE  [B, H] fp32 output (natural log).
+ *   H, Hkv       query and K/V heads, H % Hkv == 0; query head h reads K/V head
+ *                h / (H / Hkv) (as fa_fwd_gqa).
+ *   d            64 or 128;  page_size  a power of two from 8 to 4096
+ *                (FA_ERR_UNSUPPORTED otherwise).
+ *   scale        softmax scale, finite and > 0.
+ *   workspace    device buffer of workspace_bytes (16-byte aligned) or NULL.
+ *                With at least fa_decode_workspace_size() bytes, long sequences
+ *                are split into key chunks processed by separate CTAs and merged
+ *                (fp32 partials); with less, the call splits no further than the
+ *                buffer holds (NULL: one chunk per sequence).
+ * Each query attends to all seqlens[b] cached positions (the caller appends the
+ * new token's K, V before the call); a sequence with seqlens[b] == 0 gets O = 0
+ * and LSE = -inf.  Q, the pools and O must be 16-byte aligned; LSE, block_table
+ * and seqlens 4-byte aligned.  num_pages * page_size and max_pages * page_size
+ * must stay below 2^31, B <= 65535 (FA_ERR_TOO_LARGE otherwise).  Because
+ * seqlens and block_table are device data, the kernel checks them: a length
+ * out of range or a page index outside [0, num_pages) leaves the affected
+ * sequence's rows empty (O = 0, LSE = -inf), loads nothing from the pool, and
+ * makes the next fa_last_device_status() return FA_ERR_DEVICE_INPUT.
+ */
+int fa_decode_paged(const void* Q, const void* K_cache, const void* V_cache, const int* block_table,
+                    const int* seqlens, void* O, float* LSE, int B, int H, int Hkv, int d, int page_size,
+                    int num_pages, int max_pages, float scale, void* workspace, size_t workspace_bytes,
+                    void* stream);
+
+/* Workspace bytes with which fa_decode_paged splits as it would unconstrained:
+ * the fp32 partials of each key chunk (0 when one chunk suffices or the
+ * arguments are invalid). */
+size_t fa_decode_workspace_size(int B, int H, int Hkv, int d, int page_size, int max_pages);
+
 /* Static English text for a status code. */
 const char* fa_status_string(int status);
 
@@ -286,9 +331,12 @@ int fa_last_cuda_error(void);
 /*
  * Synchronises `stream`, then reads and clears the current device's status
  * word.  Returns FA_OK if no kernel reported a problem since the last call,
- * FA_ERR_DEVICE_TIMEOUT if a bounded wait expired (the affected launch's
- * outputs are then undefined), or FA_ERR_LAUNCH.  *detail (if not NULL)
- * receives the raw word: 0x1000 | the id of the wait that expired.
+ * FA_ERR_DEVICE_INPUT if a kernel found device-side input out of range
+ * (fa_decode_paged), FA_ERR_DEVICE_TIMEOUT if a bounded wait expired (the
+ * affected launch's outputs are then undefined), or FA_ERR_LAUNCH.  *detail
+ * (if not NULL) receives the raw word: 0x1000 | the id of the wait that
+ * expired, or 0x2000 | the id of the failed input check (0xD1 a sequence
+ * length, 0xD2 a page index).
  */
 int fa_last_device_status(void* stream, int* detail);
 

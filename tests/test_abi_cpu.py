@@ -46,7 +46,7 @@ def test_library_exports_every_declared_symbol(L):
 
 
 def test_status_strings(L):
-    for code in (0, -1, -2, -3, -4, -5, -6, -7, -8):
+    for code in (0, -1, -2, -3, -4, -5, -6, -7, -8, -9):
         assert fa.status_string(code) and "unknown" not in fa.status_string(code)
     assert "unknown" in fa.status_string(-99)
 
@@ -222,3 +222,48 @@ def test_blocksparse_validation(L):
     ws = L.fa_bwd_workspace_size(1, 4, 256, 128, 0)
     assert b(*args, 1, 4, 4, 256, 128, 0.1, -1, -1, None, 1, 0, 256, ws, None) == -1
     assert b(*args, 1, 4, 4, 256, 128, 0.1, -1, -1, 16, 3, 0, 256, ws, None) == -1
+
+
+def test_decode_validation(L):
+    """fa_decode_paged argument checks, all before any device work."""
+    f = L.fa_decode_paged
+    # Q, K, V, table, seqlens, O, LSE, B, H, Hkv, d, page_size, num_pages, max_pages, scale, ws, bytes, stream
+    ok = dict(B=2, H=8, Hkv=2, d=128, P=16, npg=10, mp=4, sc=0.1)
+
+    def call(ptr=16, q=None, **kw):
+        a = {**ok, **kw}
+        p = ptr if q is None else q
+        return f(p, ptr, ptr, ptr, ptr, ptr, ptr, a["B"], a["H"], a["Hkv"], a["d"], a["P"], a["npg"], a["mp"],
+                 a["sc"], None, 0, None)
+
+    assert call(ptr=None) == -1                       # null pointers
+    assert call(d=96) == -2                           # head dim
+    for p in (0, 4, 12, 48, 8192):                    # page size: a power of two in [8, 4096]
+        assert call(P=p) == -2, p
+    assert call(Hkv=3) == -1                          # grouping
+    assert call(sc=0.0) == -1 and call(sc=float("nan")) == -1
+    assert call(npg=0) == -1 and call(mp=0) == -1 and call(B=-1) == -1
+    assert call(npg=1 << 28, P=16) == -8              # pool rows beyond 2^31
+    assert call(mp=1 << 28, P=16) == -8               # table span beyond 2^31
+    assert call(B=65536) == -8
+    assert call(q=8) == -3                            # misaligned Q
+    assert call(B=0, ptr=None) == 0                   # empty batch
+    # workspace sizes: none for a full batch of short sequences, chunks for a long one
+    assert L.fa_decode_workspace_size(64, 64, 8, 128, 16, 8) == 0
+    n = L.fa_decode_workspace_size(1, 32, 8, 128, 16, 4096)
+    assert n > 0 and n % 256 == 0
+    assert L.fa_decode_workspace_size(1, 32, 8, 96, 16, 4096) == 0
+
+
+def test_python_decode_checks_shapes(L):
+    import torch
+    q = torch.zeros(2, 8, 128, dtype=torch.bfloat16)
+    k = torch.zeros(4, 16, 2, 128, dtype=torch.bfloat16)
+    t = torch.zeros(2, 2, dtype=torch.int32)
+    s = torch.zeros(2, dtype=torch.int32)
+    with pytest.raises(ValueError):
+        fa.decode_paged(q, k, k, t, s)                # CPU tensors: no CPU path
+    with pytest.raises(ValueError):
+        fa.decode_paged(q, k[..., :64], k[..., :64], t, s)
+    with pytest.raises(TypeError):
+        fa.decode_paged(q, k, k, t.long(), s)
