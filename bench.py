@@ -457,7 +457,7 @@ def run_ours(args, world, rank, local):
     out_h = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (o, lse, dq, dk, dv)]
     h2d = sum(t.numel() * t.element_size() for t in pin)
     d2h = sum(t.numel() * t.element_size() for t in out_h)
-    e_steps = max(1, min(args.steps, 10))
+    e_steps = max(1, args.steps)  # as many steps as the device-timed region: fill and drain amortise alike
     bufs = [dict(q=q, k=k, v=v, do=do, o=o, lse=lse, dq=dq, dk=dk, dv=dv)]
     bufs.append({key: torch.empty_like(t) for key, t in bufs[0].items()})
     up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)

@@ -729,16 +729,25 @@ size_t decode_ws_bytes(int B, int H, int d, int splits) {
   return align256(rows * d * sizeof(float)) + align256(rows * sizeof(float));
 }
 
-// Chunks per (sequence, head group): enough CTAs for two waves at two CTAs per SM,
-// at least four 64-key tiles per chunk, and no more than the workspace holds.
+// Chunks per (sequence, head group).  Each CTA pays a fixed start (length and
+// page checks, the first loads in flight) and end (merge of its warps), so chunks
+// hold at least 512 KB of K/V (16 tiles at d = 128, 32 at d = 64).  A batch with
+// fewer (sequence, head group) pairs than CTA slots (148 SMs x 2) is split into
+// one wave; a larger batch, whose lengths differ, into about four waves, the
+// later waves' chunks being the short or empty ends of the sequences.  No more
+// chunks than the workspace holds.
 DecodePlan decode_plan(int B, int H, int Hkv, int d, int page_size, int max_pages, size_t ws_cap) {
   DecodePlan p;
   p.hgroups = (H / Hkv + 15) / 16;
   const long long max_keys = static_cast<long long>(max_pages) * page_size;
   const long long tiles = (max_keys + 63) / 64;
   const long long ctas = static_cast<long long>(B) * Hkv * p.hgroups;
-  long long want = ctas > 0 ? (4 * 148 + ctas - 1) / ctas : 1;
-  want = std::max(1LL, std::min(want, tiles / 4));
+  const long long slots = 2 * 148;
+  const long long waves = 4;  // for batches that fill the slots
+  const long long min_tiles = d == 128 ? 16 : 32;
+  // one wave: as many chunks as fit without a second, partial wave
+  long long want = ctas <= 0 ? 1 : (ctas < slots ? slots / ctas : (waves * slots + ctas - 1) / ctas);
+  want = std::max(1LL, std::min({want, tiles / min_tiles, 65535LL}));
   for (;;) {
     const long long chunk_tiles = (tiles + want - 1) / want;
     p.splits = static_cast<int>((tiles + chunk_tiles - 1) / chunk_tiles);

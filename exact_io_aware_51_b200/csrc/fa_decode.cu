@@ -12,7 +12,7 @@
 // The step is HBM-bound: each cached K/V row is read once per (sequence, K/V
 // head) and feeds only H / Hkv query heads, 2 FLOP per byte at 8 heads.  The
 // kernel is built around moving those bytes:
-//   * grid (chunk, K/V head x head group, sequence); a CTA takes up to 16 query
+//   * grid (K/V head x head group, sequence, chunk); a CTA takes up to 16 query
 //     heads of one K/V head and one chunk of the sequence's keys (long
 //     sequences split into several chunks so small batches still fill the GPU);
 //   * one producer thread walks the chunk 64 keys at a time and, per page
@@ -113,10 +113,12 @@ __global__ void __launch_bounds__(kThreads, 2)
   DecBars* bars = reinterpret_cast<DecBars*>(smem + C::kOffBar);
   const int warp = warp_id();
   const int lane = lane_id();
-  const int split = blockIdx.x;
-  const int hkv = blockIdx.y / a.hgroups;
-  const int hg = blockIdx.y % a.hgroups;
-  const int b = blockIdx.z;
+  // chunk index slowest: the first CTAs to run take every sequence's first
+  // chunk, the later ones the (shorter, often empty) chunks further out
+  const int split = blockIdx.z;
+  const int hkv = blockIdx.x / a.hgroups;
+  const int hg = blockIdx.x % a.hgroups;
+  const int b = blockIdx.y;
   const int G = a.H / a.Hkv;
   const int h0 = hkv * G + hg * 16;      // first query head of this CTA
   const int gv = min(16, G - hg * 16);   // query heads of this CTA
@@ -363,48 +365,78 @@ __global__ void __launch_bounds__(kThreads, 2)
   }
 }
 
-// Merge of the chunks' partial results, one warp per (sequence, query head):
-// with M = max_s LSE_s and w_s = exp(LSE_s - M),
+// Merge of the chunks' partial results, one CTA of four warps per (sequence,
+// query head): with M = max_s LSE_s and w_s = exp(LSE_s - M),
 //   O = sum_s w_s O_s / sum_s w_s,   LSE = M + ln sum_s w_s.
+// The chunks are spread over the four warps (warp u takes s = u, u + 4, ...) and
+// the loads of a warp's chunks are independent, so a long sequence's many
+// partials are read with several loads in flight instead of one at a time.
 template <int D>
-__global__ void __launch_bounds__(256) decode_combine_kernel(const DecodeArgs a) {
+__global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeArgs a) {
   constexpr int kPer = D / 32;
-  const long long row = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
   const long long rows = static_cast<long long>(a.B) * a.H;
-  if (row >= rows) return;
-  const int lane = lane_id();
+  const long long row = blockIdx.x;
+  const int warp = warp_id(), lane = lane_id();
+  __shared__ float s_max[4], s_w[4];
+  __shared__ float s_acc[4][D];
   float M = -INFINITY;
-  for (int s = 0; s < a.splits; ++s) M = fmaxf(M, a.LSEpart[s * rows + row]);
+  for (int s = static_cast<int>(threadIdx.x); s < a.splits; s += 128) M = fmaxf(M, a.LSEpart[s * rows + row]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  if (lane == 0) s_max[warp] = M;
+  __syncthreads();
+  M = fmaxf(fmaxf(s_max[0], s_max[1]), fmaxf(s_max[2], s_max[3]));
   float acc[kPer];
 #pragma unroll
   for (int i = 0; i < kPer; ++i) acc[i] = 0.f;
-  float lse = -INFINITY;
+  float wsum = 0.f;
   if (M != -INFINITY) {
-    float wsum = 0.f;
-    for (int s = 0; s < a.splits; ++s) {
+#pragma unroll 4
+    for (int s = warp; s < a.splits; s += 4) {
       const float ls = a.LSEpart[s * rows + row];
-      if (ls == -INFINITY) continue;
-      const float wgt = expf(ls - M);
-      wsum += wgt;
+      const float wgt = (ls == -INFINITY) ? 0.f : expf(ls - M);
       const float* op = a.Opart + (s * rows + row) * D + lane * kPer;
+      float v[kPer];
+      if constexpr (kPer == 4) {
+        const float4 x = *reinterpret_cast<const float4*>(op);
+        v[0] = x.x;
+        v[1] = x.y;
+        v[2] = x.z;
+        v[3] = x.w;
+      } else {
+        const float2 x = *reinterpret_cast<const float2*>(op);
+        v[0] = x.x;
+        v[1] = x.y;
+      }
+      wsum += wgt;
 #pragma unroll
-      for (int i = 0; i < kPer; ++i) acc[i] += wgt * op[i];
+      for (int i = 0; i < kPer; ++i) acc[i] += wgt * v[i];
     }
-    const float inv = 1.f / wsum;
+  }
 #pragma unroll
-    for (int i = 0; i < kPer; ++i) acc[i] *= inv;
-    lse = M + logf(wsum);
+  for (int i = 0; i < kPer; ++i) s_acc[warp][lane * kPer + i] = acc[i];
+  if (lane == 0) s_w[warp] = wsum;
+  __syncthreads();
+  if (warp == 0) {
+    const float W = (s_w[0] + s_w[1]) + (s_w[2] + s_w[3]);
+    const float inv = (W > 0.f) ? 1.f / W : 0.f;
+    float out[kPer];
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+      const int c = lane * kPer + i;
+      out[i] = ((s_acc[0][c] + s_acc[1][c]) + (s_acc[2][c] + s_acc[3][c])) * inv;
+    }
+    __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.O) + row * D + lane * kPer;
+    if constexpr (kPer == 4) {
+      uint2 u;
+      u.x = pack_bf16x2(out[0], out[1]);
+      u.y = pack_bf16x2(out[2], out[3]);
+      *reinterpret_cast<uint2*>(orow) = u;
+    } else {
+      *reinterpret_cast<uint32_t*>(orow) = pack_bf16x2(out[0], out[1]);
+    }
+    if (lane == 0) a.LSE[row] = (W > 0.f) ? M + logf(W) : -INFINITY;
   }
-  __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.O) + row * D + lane * kPer;
-  if constexpr (kPer == 4) {
-    uint2 u;
-    u.x = pack_bf16x2(acc[0], acc[1]);
-    u.y = pack_bf16x2(acc[2], acc[3]);
-    *reinterpret_cast<uint2*>(orow) = u;
-  } else {
-    *reinterpret_cast<uint32_t*>(orow) = pack_bf16x2(acc[0], acc[1]);
-  }
-  if (lane == 0) a.LSE[row] = lse;
 }
 
 template <int D>
@@ -413,11 +445,11 @@ cudaError_t launch_decode_d(const CUtensorMap& tk, const CUtensorMap& tv, const 
   using C = DecCfg<D>;
   cudaError_t e = cudaFuncSetAttribute(decode_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
-  const dim3 grid(a.splits, a.Hkv * a.hgroups, a.B);
+  const dim3 grid(a.Hkv * a.hgroups, a.B, a.splits);
   decode_kernel<D><<<grid, kThreads, C::kSmemBytes, s>>>(tk, tv, a, c);
   if ((e = cudaGetLastError()) != cudaSuccess || a.splits == 1) return e;
   const long long rows = static_cast<long long>(a.B) * a.H;
-  decode_combine_kernel<D><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, s>>>(a);
+  decode_combine_kernel<D><<<static_cast<unsigned>(rows), 128, 0, s>>>(a);
   return cudaGetLastError();
 }
 
