@@ -40,60 +40,91 @@ __device__ __forceinline__ uint4 pack8(const float* f) {
   return u;
 }
 
-// One thread per 8 features of one (b, n, h) row; the d / 8 threads of a row are
-// consecutive lanes of one warp.  Every lane runs the same number of loop trips
-// (inactive lanes are predicated off), so the warp can meet at __syncwarp()
-// between reading the row's old LSE and its first lane writing the new one.
+// One thread per 8 features of one (b, n, h) row; the D / 8 threads of a row are
+// consecutive lanes of one warp.  A warp takes kRows = 2 x 32 / (D / 8) rows per
+// trip, issuing the loads of both halves before any arithmetic so twice the
+// bytes are in flight.  Trips are per warp, so every lane runs the same number
+// and the warp can meet at __syncwarp() between reading the rows' old LSE and
+// writing the new one.  Idx is 32-bit whenever B N H d fits, so the
+// row -> (b, n, h) split costs a few integer instructions rather than 64-bit
+// divisions.
+template <int D, typename Idx>
 __global__ void __launch_bounds__(kThreads)
     merge_kernel(float* __restrict__ o_acc, float* __restrict__ lse_acc, const __nv_bfloat16* __restrict__ o_part,
-                 const float* __restrict__ lse_part, __nv_bfloat16* __restrict__ o_out, int B, int H, int N, int d,
+                 const float* __restrict__ lse_part, __nv_bfloat16* __restrict__ o_out, int B, int H, int N,
                  int init) {
-  const int per_row = d / 8;
-  const long long total = static_cast<long long>(B) * N * H * per_row;
-  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
-  for (long long base = static_cast<long long>(blockIdx.x) * blockDim.x; base < total; base += stride) {
-    const long long idx = base + threadIdx.x;
-    const bool active = idx < total;
-    const long long row = active ? idx / per_row : 0;  // (b, n, h) in [B, N, H] order
-    const int part = static_cast<int>(idx % per_row);
-    const int h = static_cast<int>(row % H);
-    const long long bn = row / H;
-    const int n = static_cast<int>(bn % N);
-    const int b = static_cast<int>(bn / N);
-    const size_t li = (static_cast<size_t>(b) * H + h) * N + n;
-    const size_t oi = static_cast<size_t>(row) * d + part * 8;
-    float o[8], l = -INFINITY;
-    if (active) {
-      float ob[8];
-      unpack8(*reinterpret_cast<const uint4*>(o_part + oi), ob);
-      const float lb = lse_part[li];
+  constexpr int kPerRow = D / 8;
+  constexpr int kRowsPerHalf = 32 / kPerRow;
+  constexpr int kRows = 2 * kRowsPerHalf;
+  const Idx rows = static_cast<Idx>(B) * N * H;
+  const int lane = threadIdx.x & 31;
+  const int part = lane % kPerRow;
+  const Idx nwarps = static_cast<Idx>(gridDim.x) * (kThreads / 32);
+  for (Idx r0 = (static_cast<Idx>(blockIdx.x) * (kThreads / 32) + threadIdx.x / 32) * kRows; r0 < rows;
+       r0 += nwarps * kRows) {
+    bool active[2];
+    Idx li[2], oi[2];
+    uint4 pb[2];
+    float4 a0[2], a1[2];
+    float la[2], lb[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const Idx row = r0 + u * kRowsPerHalf + lane / kPerRow;  // (b, n, h) in [B, N, H] order
+      active[u] = row < rows;
+      const Idx h = row % static_cast<Idx>(H);
+      const Idx bn = row / static_cast<Idx>(H);
+      const Idx n = bn % static_cast<Idx>(N);
+      const Idx b = bn / static_cast<Idx>(N);
+      li[u] = (b * H + h) * N + n;
+      oi[u] = row * D + part * 8;
+      la[u] = -INFINITY;
+      lb[u] = -INFINITY;
+      pb[u] = make_uint4(0u, 0u, 0u, 0u);
+      a0[u] = a1[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (active[u]) {
+        pb[u] = *reinterpret_cast<const uint4*>(o_part + oi[u]);
+        lb[u] = lse_part[li[u]];
+        if (!init) {
+          la[u] = lse_acc[li[u]];
+          a0[u] = *reinterpret_cast<const float4*>(o_acc + oi[u]);
+          a1[u] = *reinterpret_cast<const float4*>(o_acc + oi[u] + 4);
+        }
+      }
+    }
+    float l[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      float o[8], ob[8];
+      unpack8(pb[u], ob);
+      const float oa[8] = {a0[u].x, a0[u].y, a0[u].z, a0[u].w, a1[u].x, a1[u].y, a1[u].z, a1[u].w};
+      l[u] = -INFINITY;
       if (init) {
 #pragma unroll
         for (int i = 0; i < 8; ++i) o[i] = ob[i];
-        l = lb;
+        l[u] = lb[u];
       } else {
-        const float la = lse_acc[li];
-        const float4 a0 = *reinterpret_cast<const float4*>(o_acc + oi);
-        const float4 a1 = *reinterpret_cast<const float4*>(o_acc + oi + 4);
-        const float oa[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-        const float m = fmaxf(la, lb);
+        const float m = fmaxf(la[u], lb[u]);
         if (m == -INFINITY) {  // neither part saw a key
 #pragma unroll
           for (int i = 0; i < 8; ++i) o[i] = 0.f;
         } else {
-          const float wa = expf(la - m), wb = expf(lb - m);
+          const float wa = expf(la[u] - m), wb = expf(lb[u] - m);
           const float inv = 1.f / (wa + wb);
 #pragma unroll
           for (int i = 0; i < 8; ++i) o[i] = (wa * oa[i] + wb * ob[i]) * inv;
-          l = m + logf(wa + wb);
+          l[u] = m + logf(wa + wb);
         }
       }
-      *reinterpret_cast<float4*>(o_acc + oi) = make_float4(o[0], o[1], o[2], o[3]);
-      *reinterpret_cast<float4*>(o_acc + oi + 4) = make_float4(o[4], o[5], o[6], o[7]);
-      if (o_out) *reinterpret_cast<uint4*>(o_out + oi) = pack8(o);
+      if (active[u]) {
+        *reinterpret_cast<float4*>(o_acc + oi[u]) = make_float4(o[0], o[1], o[2], o[3]);
+        *reinterpret_cast<float4*>(o_acc + oi[u] + 4) = make_float4(o[4], o[5], o[6], o[7]);
+        if (o_out) *reinterpret_cast<uint4*>(o_out + oi[u]) = pack8(o);
+      }
     }
-    __syncwarp();  // every lane of the row has read lse_acc[li]
-    if (active && part == 0) lse_acc[li] = l;
+    __syncwarp();  // every lane of the warp's rows has read lse_acc
+#pragma unroll
+    for (int u = 0; u < 2; ++u)
+      if (active[u] && part == 0) lse_acc[li[u]] = l[u];
   }
 }
 
@@ -135,12 +166,20 @@ unsigned grid_for(long long items) {
 
 cudaError_t launch_merge(float* o_acc, float* lse_acc, const void* o_part, const float* lse_part, void* o_out, int B,
                          int H, int N, int d, int init, cudaStream_t s) {
-  // per_row = d / 8 (8 or 16) divides 32, so the threads of one row are lanes of one warp
   static_assert(kThreads % 32 == 0, "whole warps");
   if (d != 64 && d != 128) return cudaErrorInvalidValue;
-  const long long items = static_cast<long long>(B) * N * H * (d / 8);
-  merge_kernel<<<grid_for(items), kThreads, 0, s>>>(o_acc, lse_acc, static_cast<const __nv_bfloat16*>(o_part), lse_part,
-                                                    static_cast<__nv_bfloat16*>(o_out), B, H, N, d, init);
+  const long long rows = static_cast<long long>(B) * N * H;
+  const unsigned grid = grid_for(rows * (d / 8));
+  const bool narrow = rows * d < (1LL << 32);
+  auto p = static_cast<const __nv_bfloat16*>(o_part);
+  auto q = static_cast<__nv_bfloat16*>(o_out);
+  if (d == 128) {
+    if (narrow) merge_kernel<128, uint32_t><<<grid, kThreads, 0, s>>>(o_acc, lse_acc, p, lse_part, q, B, H, N, init);
+    else merge_kernel<128, unsigned long long><<<grid, kThreads, 0, s>>>(o_acc, lse_acc, p, lse_part, q, B, H, N, init);
+  } else {
+    if (narrow) merge_kernel<64, uint32_t><<<grid, kThreads, 0, s>>>(o_acc, lse_acc, p, lse_part, q, B, H, N, init);
+    else merge_kernel<64, unsigned long long><<<grid, kThreads, 0, s>>>(o_acc, lse_acc, p, lse_part, q, B, H, N, init);
+  }
   return cudaGetLastError();
 }
 
