@@ -732,10 +732,10 @@ size_t decode_ws_bytes(int B, int H, int d, int splits) {
 // Chunks per (sequence, head group).  Each CTA pays a fixed start (length and
 // page checks, the first loads in flight) and end (merge of its warps), so chunks
 // hold at least 512 KB of K/V (16 tiles at d = 128, 32 at d = 64).  A batch with
-// fewer (sequence, head group) pairs than CTA slots (148 SMs x 2) is split to
-// fill one wave (at least three chunks per sequence); a larger batch into about
-// four waves, the later waves' chunks being the short or empty ends of the
-// sequences.  No more chunks than the workspace holds.
+// fewer (sequence, head group) pairs than CTA slots (148 SMs x 2) is split into
+// about two waves of CTAs; a larger batch into about four, the later waves'
+// chunks being the short or empty ends of the sequences.  No more chunks than
+// the workspace holds.
 DecodePlan decode_plan(int B, int H, int Hkv, int d, int page_size, int max_pages, size_t ws_cap) {
   DecodePlan p;
   p.hgroups = (H / Hkv + 15) / 16;
@@ -745,9 +745,10 @@ DecodePlan decode_plan(int B, int H, int Hkv, int d, int page_size, int max_page
   const long long slots = 2 * 148;
   const long long waves = 4;  // for batches that fill the slots
   const long long min_tiles = d == 128 ? 16 : 32;
-  // a small batch: as many chunks as fill one wave, but at least three per
-  // sequence so that one long sequence among short ones is not a lone tail
-  long long want = ctas <= 0 ? 1 : (ctas < slots ? std::max(slots / ctas, 3LL) : (waves * slots + ctas - 1) / ctas);
+  // a small batch: two waves (one wave suits equal lengths best, but a long
+  // sequence among shorter ones then runs alone at the end)
+  const long long w = ctas < slots ? 2 : waves;
+  long long want = ctas <= 0 ? 1 : (w * slots + ctas - 1) / ctas;
   want = std::max(1LL, std::min({want, tiles / min_tiles, 65535LL}));
   for (;;) {
     const long long chunk_tiles = (tiles + want - 1) / want;
