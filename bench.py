@@ -63,6 +63,15 @@ def read_peaks():
     return FALLBACK_PEAK_TFLOPS, 1400.0, "fallback"
 
 
+def choose_peak(clocks: dict, burst: float, sustained: float):
+    """The tensor peak a kernel timed inside the step loop is compared with: the
+    sustained cuBLAS figure when the clock record shows the power cap active over
+    the timed steps (both then run at the cap), else the burst one."""
+    if "sw_power_cap" in (clocks.get("reasons") or []):
+        return sustained, "sustained (cuBLAS loop at the power cap; the timed steps ran at the cap)"
+    return burst, "burst"
+
+
 def read_hbm_peak():
     p = ROOT / "MEASURED_PEAKS.json"
     if p.exists():
@@ -374,9 +383,7 @@ def run_ours(args, world, rank, local):
     # record shows the power cap active over that region, the comparable peak is
     # the sustained cuBLAS figure (a GEMM loop held at the same cap); otherwise
     # the burst one.  Both fractions are reported.
-    capped = "sw_power_cap" in (clocks.get("reasons") or [])
-    peak = peak_sustained if capped else peak_burst
-    peak_kind = "sustained (cuBLAS loop at the power cap; the timed steps ran at the cap)" if capped else "burst"
+    peak, peak_kind = choose_peak(clocks, peak_burst, peak_sustained)
     roofline = {"bound": "tensor", "kernel": dom["kernel"], "achieved": achieved, "peak": peak,
                 "peak_source": f"{peak_src} bf16 {peak_kind}", "unit": "TFLOP/s", "frac": achieved / peak,
                 "frac_of_burst": achieved / peak_burst,

@@ -72,3 +72,33 @@ def test_reference_arm_on_a_non_zero_rank_exits_quietly():
                         "--steps", "1", "--warmup", "0"], capture_output=True, text=True, env=env, timeout=300)
     assert r.returncode == 0, r.stderr
     assert r.stdout.strip() == ""
+
+
+def test_peak_follows_the_power_state_of_the_timed_steps():
+    """Kernels timed while the power cap is active are compared with the sustained
+    GEMM figure; otherwise with the burst one."""
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.choose_peak({"reasons": ["sw_power_cap"]}, 1660.9, 1397.6)[0] == 1397.6
+    assert bench.choose_peak({"reasons": []}, 1660.9, 1397.6)[0] == 1660.9
+    assert bench.choose_peak({"reasons": None}, 1660.9, 1397.6)[0] == 1660.9
+    assert bench.choose_peak({}, 1660.9, 1397.6)[0] == 1660.9
+
+
+def test_nvml_sampler_keeps_only_the_marked_window():
+    """Samples outside [mark_begin, mark_end] are dropped; no samples gives None."""
+    sys.path.insert(0, ROOT)
+    import bench
+    s = bench.NvmlSampler(0)
+
+    class _T:  # stands in for the sampling thread that ran
+        def join(self, timeout=None):
+            return None
+    s.thread = _T()
+    s.max_mhz = 1965
+    s.begin, s.end = 10.0, 20.0
+    s.rows = [(5.0, 1965, 300.0, 0), (12.0, 1700, 900.0, 0x4), (15.0, 1690, 950.0, 0x4), (25.0, 1965, 200.0, 0)]
+    r = s.stop()
+    assert r["samples"] == 2 and r["sm_mhz"] == 1695 and r["reasons"] == ["sw_power_cap"]
+    s2 = bench.NvmlSampler(0)
+    assert s2.stop() is None
