@@ -9,21 +9,28 @@
 //   dV = P^T dO,  dP = dO V^T,  D_i = sum_k dO_ik O_ik,  dS = P * (dP - D),
 //   dQ = scale * dS K,  dK = scale * dS^T Q.
 //
-// Three kernels on one stream:
+// Three kernels on one stream (four more with a split walk, see below):
 //   1. bwd_pre:  D_i = rowsum(dO * O) and L_i * log2(e) into [B, H, Npad]
 //      fp32 rows, and zero the fp32 dQ accumulator (HBM-bound);
-//   2. bwd_main: one CTA per 128-key tile j of one (b, h).  K_j and V_j stay in
-//      shared memory; 64-row query tiles i stream past through a TMA ring.
-//      Per tile, five tcgen05 MMAs with TMEM accumulators:
-//        S^T  = K_j Q_i^T          (keys on TMEM lanes)
+//   2. bwd_main: one CTA per 128-key tile j of one (b, K/V head).  K_j and V_j
+//      stay in shared memory; 128-row query tiles i (of every query head of
+//      the K/V head's group) stream past through a 2-stage TMA ring.  Per tile,
+//      five tcgen05 MMAs with TMEM accumulators:
+//        S^T  = K_j Q_i^T          (keys on TMEM lanes; both operands in smem)
 //        dP^T = V_j dO_i^T
-//        dV_j += P^T dO_i          (P^T written by the softmax warps to smem)
-//        dK_j += dS^T Q_i          (dS^T likewise)
-//        dQ_i^T = K_j^T dS^T       (features on TMEM lanes, double buffered)
-//      One warpgroup turns S^T / dP^T into P^T / dS^T (one key row per thread,
-//      exp2 with the scale folded in), one warpgroup drains dQ_i^T from TMEM
-//      into the fp32 accumulator with coalesced reductions, one warp loads and
-//      one warp issues MMAs.  Causal: query tiles above the diagonal are skipped.
+//        dV_j += P^T dO_i          (P^T written over S^T in TMEM as bf16 pairs)
+//        dK_j += dS^T Q_i          (dS^T written over dP^T in TMEM likewise)
+//        dQ_i^T = K_j^T dS^T       (features on TMEM lanes; dS^T also stored to
+//                                   smem over dO_i as the B operand)
+//      Two warpgroups turn S^T / dP^T into P^T / dS^T (one key row per thread,
+//      64 query columns each, exp2 with the scale folded in); one warpgroup
+//      reads dQ_i^T out of TMEM, stages 64 query rows at a time in shared
+//      memory and adds them into the fp32 accumulator with TMA reduce-adds;
+//      one warp loads and one warp issues MMAs.  Causal, window and
+//      block-sparse masks: query tiles no key of the tile can see are skipped.
+//      Small grids split each key tile's walk over several CTAs, whose fp32
+//      dK, dV partial sums are added into workspace accumulators (zeroed before
+//      and converted to bf16 after the main kernel).
 //   3. bwd_dq:   dQ = bf16(scale * dQacc).
 #include <cuda_bf16.h>
 
