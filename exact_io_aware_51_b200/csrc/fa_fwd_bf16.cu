@@ -27,6 +27,11 @@
 //     (karlkratz.de), "Sliding Window Attention": blocks outside the window
 //     are skipped); only the tiles that straddle the window's edge are masked;
 //     under the causal mask CTAs with longer rows start first;
+//   * block-sparse masks (the kSparse instantiation): the CTA compacts the key
+//     tiles either query tile keeps into a list in shared memory; the loader
+//     streams only those, and each tile skips the ones it does not keep; a
+//     row that keeps none gets O = 0, LSE = -inf;
+//   * grouped-query attention: query head h reads K/V head h / (H / Hkv);
 //   * epilogue: O / l -> bf16 with 16-byte stores, LSE = (m + log2 l) ln 2.
 // The two query tiles ping-pong: while the softmax of one tile runs, the
 // tensor pipe computes the other tile's products.
