@@ -359,10 +359,11 @@ int fa_last_device_status(void* stream, int* detail) {
 
 namespace {
 // Block-sparse mask checks: mask_heads is 1 or H and the key-tile count fits the
-// kernels' per-CTA list.  A null mask means no mask.
+// kernels' per-CTA list.  A null mask means no mask.  (Both dtypes take a mask in
+// the forward; the backward refuses fp32 on its own.)
 int check_mask(const uint8_t* mask, int mask_heads, int H, int N, int dtype) {
+  (void)dtype;
   if (!mask) return FA_OK;
-  if (dtype != FA_BF16) return FA_ERR_UNSUPPORTED;
   if (mask_heads != 1 && mask_heads != H) return FA_ERR_INVALID_ARG;
   if ((N + 127) / 128 > kMaxSparseTiles) return FA_ERR_TOO_LARGE;
   return FA_OK;

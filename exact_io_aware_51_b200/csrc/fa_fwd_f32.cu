@@ -10,7 +10,11 @@
 //
 // Layout: one CTA per 128 query rows of one (b, h); each row is owned by
 // D / 64 threads (each holds 64 features of q and of the output accumulator);
-// 32-key K/V tiles are staged in shared memory and read as broadcasts.
+// 32-key K/V tiles are staged in shared memory and read as broadcasts.  The
+// CTA's 128 rows are exactly one block of a block-sparse mask, so a key tile
+// whose 128-key block the mask drops is skipped by the whole CTA ("Flash
+// Attention" (Ultralytics glossary), "Flash Attention и смежные понятия": the
+// block-sparse form skips empty blocks).
 #include "fa_internal.h"
 
 namespace fa {
@@ -53,7 +57,13 @@ __global__ void __launch_bounds__(kRows * (D / 64))
   // keys some row of this CTA may see: [first_key, last_key)
   const int first_key = max(0, row0 - a.wl) / kKT * kKT;
   const int last_key = min(a.N - 1, row0 + kRows - 1 + a.wr) + 1;
+  // this query block's row of the block mask (null: every block kept)
+  const uint8_t* mrow =
+      a.block_mask ? a.block_mask + (static_cast<size_t>(a.mask_heads == 1 ? 0 : h) * a.nb + blockIdx.x) * a.nb
+                   : nullptr;
+  static_assert(kRows == 128 && 128 % kKT == 0, "a CTA's rows form one mask block; a key tile lies in one");
   for (int k0 = first_key; k0 < last_key; k0 += kKT) {
+    if (mrow && mrow[k0 / 128] == 0) continue;  // the same for every thread of the CTA
     __syncthreads();
     for (int e = tid * 4; e < kKT * D; e += kThreads * 4) {
       const int kr = e / D, kc = e % D;

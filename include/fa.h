@@ -123,8 +123,8 @@ int fa_fwd_window(const void* Q, const void* K, const void* V, void* O, float* L
  *   mask_heads  1 or H (FA_ERR_INVALID_ARG otherwise).
  *   window_left, window_right  as fa_fwd_window; both masks apply.
  * Key blocks a query block does not see are neither loaded nor multiplied.  A
- * row that sees no key gets O = 0 and LSE = -inf.  bf16 only
- * (FA_ERR_UNSUPPORTED for FA_FP32); nb <= 4096, i.e. N <= 524288
+ * row that sees no key gets O = 0 and LSE = -inf.  FA_BF16 (tensor cores) and
+ * FA_FP32 (the exact fp32 kernel); nb <= 4096, i.e. N <= 524288
  * (FA_ERR_TOO_LARGE otherwise).  Other arguments as fa_fwd_window.
  */
 int fa_fwd_blocksparse(const void* Q, const void* K, const void* V, void* O, float* LSE, int B, int H, int Hkv,

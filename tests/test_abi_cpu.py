@@ -213,7 +213,7 @@ def test_blocksparse_validation(L):
     # null mask, wrong mask_heads, fp32, too many key blocks
     assert f(16, 16, 16, 16, 16, 1, 4, 4, 256, 128, 0.1, -1, -1, None, 1, 0, None) == -1
     assert f(16, 16, 16, 16, 16, 1, 4, 4, 256, 128, 0.1, -1, -1, 16, 2, 0, None) == -1
-    assert f(16, 16, 16, 16, 16, 1, 4, 4, 256, 128, 0.1, -1, -1, 16, 1, 1, None) == -2
+    assert f(8, 16, 16, 16, 16, 1, 4, 4, 256, 128, 0.1, -1, -1, 16, 1, 1, None) == -3  # fp32 passes the dtype check
     assert f(16, 16, 16, 16, 16, 1, 4, 4, 4096 * 128 + 1, 128, 0.1, -1, -1, 16, 1, 0, None) == -8
     # valid arguments reach the alignment check
     assert f(8, 16, 16, 16, 16, 1, 4, 4, 256, 128, 0.1, -1, -1, 16, 4, 0, None) == -3

@@ -19,7 +19,7 @@ import torch
 import exact_io_aware_51_b200 as fa
 import oracle
 from exact_io_aware_51_b200 import inputs as I
-from tests.helpers import TOL_BF16_REL, TOL_LSE, need_gpu, rel_err
+from tests.helpers import TOL_BF16_REL, TOL_F32_O, TOL_LSE, abs_err, need_gpu, rel_err
 
 
 def _scale(d):
@@ -57,6 +57,24 @@ def test_blocksparse_forward(n, d, heads_mask):
     ro, rl = oracle.forward(q, k, v, _scale(d), False, block_mask=m)
     assert rel_err(o.cpu(), ro) <= TOL_BF16_REL
     assert _lse_close(lse.cpu(), rl)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("n,d", [(256, 64), (333, 128), (700, 64)])
+@pytest.mark.parametrize("heads_mask", [1, 2])
+def test_blocksparse_forward_fp32(n, d, heads_mask):
+    """The exact fp32 forward under a block mask: every element within 1e-5,
+    including a block row that sees nothing (O = 0, LSE = -inf)."""
+    need_gpu()
+    nb = (n + 127) // 128
+    m = _mask(nb, heads_mask, 0.5, 7 * n + heads_mask, empty_row=nb - 1)
+    q, k, v, _ = I.make_inputs(1, n, 2, d, seed=n + 1, dtype="fp32", with_do=False)
+    o, lse = fa.fwd(q.cuda(), k.cuda(), v.cuda(), scale=_scale(d), block_mask=torch.from_numpy(m).cuda())
+    torch.cuda.synchronize()
+    ro, rl = oracle.forward(q, k, v, _scale(d), False, block_mask=m)
+    assert abs_err(o.cpu(), ro) <= TOL_F32_O
+    assert _lse_close(lse.cpu(), rl)
+    assert fa.last_device_status()[0] == 0
 
 
 @pytest.mark.gpu
