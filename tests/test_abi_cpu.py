@@ -267,3 +267,24 @@ def test_python_decode_checks_shapes(L):
         fa.decode_paged(q, k[..., :64], k[..., :64], t, s)
     with pytest.raises(TypeError):
         fa.decode_paged(q, k, k, t.long(), s)
+
+
+def test_header_is_plain_c_and_links(L, tmp_path):
+    """include/fa.h compiles as C99 and a C program linked against libfa.so calls
+    the ABI (static-text and host-only entry points; no GPU needed)."""
+    src = tmp_path / "use_fa.c"
+    src.write_text(
+        '#include <stdio.h>\n#include "fa.h"\n'
+        "int main(void) {\n"
+        "  const char* s = fa_status_string(FA_ERR_WORKSPACE);\n"
+        "  size_t ws = fa_bwd_workspace_size(1, 2, 256, 128, FA_BF16);\n"
+        "  size_t dws = fa_decode_workspace_size(1, 32, 8, 128, 16, 4096);\n"
+        '  printf("%d %s %zu %zu\\n", fa_version(), s, ws, dws);\n'
+        "  return (s && ws > 0 && dws > 0) ? 0 : 1;\n"
+        "}\n")
+    exe = tmp_path / "use_fa"
+    lib_dir = fa.lib_path().parent
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-I", str(HEADER.parent), str(src), "-o", str(exe),
+                    "-L", str(lib_dir), "-lfa", f"-Wl,-rpath,{lib_dir}"], check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()
+    assert out[0] == str(L.fa_version())
