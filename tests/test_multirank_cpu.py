@@ -102,3 +102,21 @@ def test_nvml_sampler_keeps_only_the_marked_window():
     assert r["samples"] == 2 and r["sm_mhz"] == 1695 and r["reasons"] == ["sw_power_cap"]
     s2 = bench.NvmlSampler(0)
     assert s2.stop() is None
+
+
+def test_reference_arm_prints_the_contract_line():
+    """Rank 0 of the reference arm (the CPU oracle) prints one JSON line with the
+    keys the bench contract asks for, its own e2e object and a cpu_baseline."""
+    import json
+    env = dict(os.environ, RANK="0", LOCAL_RANK="0", WORLD_SIZE="1", MASTER_ADDR="127.0.0.1")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--steps", "1", "--warmup", "0"], capture_output=True, text=True, env=env, timeout=600)
+    assert r.returncode == 0, r.stderr
+    lines = [x for x in r.stdout.splitlines() if x.startswith("{")]
+    assert len(lines) == 1
+    j = json.loads(lines[0])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "impl", "cpu_baseline", "e2e"):
+        assert key in j, key
+    assert j["impl"] == "reference" and j["value"] > 0 and j["cpu_baseline"]["kind"] == "oracle"
+    assert j["e2e"]["h2d_bytes_per_step"] == 0 and j["e2e"]["value"] == j["value"]
