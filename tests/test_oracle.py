@@ -830,3 +830,29 @@ def test_paged_decode_mutants_are_caught(kind):
             worst = math.inf  # the mistake reads outside the pool or table
     assert worst > 1e-6
     assert pin_paged_sdpa(decode=_mut_paged("none")) < 1e-12
+
+
+def test_paged_decode_randomised_tables():
+    """Random batches, page sizes, lengths and page orders (seeded): the paged
+    oracle equals torch SDPA on each sequence's contiguous rows."""
+    rng = np.random.default_rng(2024)
+    for trial in range(12):
+        B = int(rng.integers(1, 5))
+        Hkv = int(rng.choice([1, 2, 3]))
+        H = Hkv * int(rng.choice([1, 2, 4]))
+        P = int(rng.choice([1, 2, 3, 5, 8]))
+        lens = [int(x) for x in rng.integers(0, 23, size=B)]
+        if max(lens) == 0:
+            lens[0] = 1
+        q, ks, vs, kc, vc, table, lens_a = _paged_case(100 + trial, lens, H=H, Hkv=Hkv, d=4, P=P,
+                                                         spare=int(rng.integers(0, 4)))
+        o, lse = A.decode_paged(q, kc, vc, table, lens_a, 0.8)
+        for b, n in enumerate(lens):
+            if n == 0:
+                assert np.all(o[b] == 0) and np.all(np.isneginf(lse[b]))
+                continue
+            tq = torch.tensor(q[b][:, None, :])
+            tk = torch.tensor(ks[b].transpose(1, 0, 2))
+            tv = torch.tensor(vs[b].transpose(1, 0, 2))
+            ref = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, scale=0.8, enable_gqa=True)
+            assert np.max(np.abs(o[b] - ref[:, 0].numpy())) < 1e-12
