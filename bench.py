@@ -81,7 +81,8 @@ def read_hbm_peak():
 
 def read_profile_traffic(kernel_key: str):
     """DRAM bytes per launch from the committed ncu summary, if it matches the current source."""
-    prof = ROOT / "profiles" / f"{kernel_key}.md"
+    prof = ROOT / "profiles" / {"fwd_bf16": "fwd_bf16_b1_h32_n16384_d128.md",
+                                "bwd_main": "bwd_main_b1_h32_n16384_d128.md"}[kernel_key]
     if not prof.exists():
         return None
     text = prof.read_text()
