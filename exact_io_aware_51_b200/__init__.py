@@ -37,7 +37,8 @@ EXPORTED = ("fa_fwd", "fa_bwd_workspace_size", "fa_bwd", "fa_status_string", "fa
             "fa_version", "fa_set_kernel_events", "fa_bwd_static_scratch", "fa_fwd_gqa", "fa_bwd_gqa",
             "fa_fwd_window", "fa_bwd_window", "fa_debug_umma_f8", "fa_fwd_fp8",
             "fa_fwd_blocksparse", "fa_bwd_blocksparse", "fa_merge_partial", "fa_accumulate_bf16",
-            "fa_cast_bf16", "fa_bwd_workspace_size_gqa", "fa_decode_paged", "fa_decode_workspace_size")
+            "fa_cast_bf16", "fa_bwd_workspace_size_gqa", "fa_decode_paged", "fa_decode_workspace_size",
+            "fa_fwd_fp8_blocksparse")
 
 
 class FAError(RuntimeError):
@@ -79,6 +80,8 @@ def lib() -> ctypes.CDLL:
     L.fa_bwd_gqa.restype = i
     L.fa_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, f, f, f, i, i, vp]
     L.fa_fwd_fp8.restype = i
+    L.fa_fwd_fp8_blocksparse.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, f, f, f, i, i, vp, i, vp]
+    L.fa_fwd_fp8_blocksparse.restype = i
     L.fa_fwd_blocksparse.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp, i, i, vp]
     L.fa_fwd_blocksparse.restype = i
     L.fa_bwd_blocksparse.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp, i, i, vp, sz, vp]
@@ -222,9 +225,10 @@ def fwd(q, k, v, causal: bool = False, scale: float | None = None, out=None, lse
 
 
 def fwd_fp8(q, k, v, scale_q: float, scale_k: float, scale_v: float, causal: bool = False,
-            scale: float | None = None, window=None, out=None, lse=None, stream=None):
+            scale: float | None = None, window=None, out=None, lse=None, stream=None, block_mask=None):
     """Forward with 8-bit inputs: q [B, N, H, 128], k, v [B, N, Hkv, 128] as torch.float8_e4m3fn
-    (or their uint8 codes), each dequantised by its scale; returns (o bf16, lse fp32)."""
+    (or their uint8 codes), each dequantised by its scale; returns (o bf16, lse fp32).
+    ``block_mask`` as in ``fwd`` (fa_fwd_fp8_blocksparse)."""
     for t in (q, k, v):
         if t.dtype not in (torch.float8_e4m3fn, torch.uint8):
             raise TypeError("fwd_fp8 takes torch.float8_e4m3fn (or uint8 e4m3 codes)")
@@ -233,11 +237,12 @@ def fwd_fp8(q, k, v, scale_q: float, scale_k: float, scale_v: float, causal: boo
     o = torch.empty((B, N, H, d), dtype=torch.bfloat16, device=q.device) if out is None else out
     l = torch.empty((B, H, N), dtype=torch.float32, device=q.device) if lse is None else lse
     wl, wr = _window_bounds(causal, (None, None) if window is None else window)
-    rc = lib().fa_fwd_fp8(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), l.data_ptr(), B, H, Hkv, N, d,
-                          _scale(scale, d), float(scale_q), float(scale_k), float(scale_v), wl, wr,
-                          _stream_handle(stream, q.device))
+    mp, mh = _mask_args(block_mask, q) if block_mask is not None else (None, 0)
+    rc = lib().fa_fwd_fp8_blocksparse(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), l.data_ptr(), B, H,
+                                      Hkv, N, d, _scale(scale, d), float(scale_q), float(scale_k), float(scale_v),
+                                      wl, wr, mp, mh, _stream_handle(stream, q.device))
     if rc != 0:
-        raise FAError(rc, "fa_fwd_fp8")
+        raise FAError(rc, "fa_fwd_fp8_blocksparse")
     return o, l
 
 

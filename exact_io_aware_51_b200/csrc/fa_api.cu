@@ -443,14 +443,16 @@ int fa_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, int
   return fa_fwd_window(Q, K, V, O, LSE, B, H, H, N, d, scale, -1, causal ? 0 : -1, dtype, stream);
 }
 
-int fa_fwd_fp8(const void* Q, const void* K, const void* V, void* O, float* LSE, int B, int H, int Hkv, int N, int d,
-               float scale, float scale_q, float scale_k, float scale_v, int window_left, int window_right,
-               void* stream) {
+int fa_fwd_fp8_blocksparse(const void* Q, const void* K, const void* V, void* O, float* LSE, int B, int H, int Hkv,
+                           int N, int d, float scale, float scale_q, float scale_k, float scale_v, int window_left,
+                           int window_right, const void* block_mask, int mask_heads, void* stream) {
   int rc = check_shape(B, H, N, d, FA_BF16);
   if (rc) return rc;
   if (d != 128) return FA_ERR_UNSUPPORTED;
   if ((rc = check_kv_heads(H, Hkv))) return rc;
   if ((rc = check_window(window_left, window_right))) return rc;
+  const uint8_t* mask = static_cast<const uint8_t*>(block_mask);
+  if ((rc = check_mask(mask, mask_heads, H, N, FA_BF16))) return rc;
   if ((rc = check_scale(scale)) || (rc = check_scale(scale_q)) || (rc = check_scale(scale_k)) ||
       (rc = check_scale(scale_v)))
     return rc;
@@ -471,8 +473,8 @@ int fa_fwd_fp8(const void* Q, const void* K, const void* V, void* O, float* LSE,
   set_window(window_left, window_right, &a.wl, &a.wr, &a.causal);
   a.O = O;
   a.LSE = LSE;
-  a.block_mask = nullptr;
-  a.mask_heads = 0;
+  a.block_mask = mask;
+  a.mask_heads = mask ? mask_heads : 0;
   a.nb = (N + 127) / 128;
   CUtensorMap tq, tk, tv;
   CUresult r;
@@ -485,6 +487,13 @@ int fa_fwd_fp8(const void* Q, const void* K, const void* V, void* O, float* LSE,
   if (e != cudaSuccess) return fail_cuda(e);
   if (t_ev_stop) cudaEventRecord(t_ev_stop, s);
   return FA_OK;
+}
+
+int fa_fwd_fp8(const void* Q, const void* K, const void* V, void* O, float* LSE, int B, int H, int Hkv, int N, int d,
+               float scale, float scale_q, float scale_k, float scale_v, int window_left, int window_right,
+               void* stream) {
+  return fa_fwd_fp8_blocksparse(Q, K, V, O, LSE, B, H, Hkv, N, d, scale, scale_q, scale_k, scale_v, window_left,
+                                window_right, nullptr, 0, stream);
 }
 
 size_t fa_bwd_workspace_size_gqa(int B, int H, int Hkv, int N, int d, int dtype) {

@@ -55,6 +55,8 @@ struct Cfg {
   static constexpr int kOffV = kOffK + kStages * kTile;
   static constexpr int kOffBar = kOffV + kStages * kTile;
   static constexpr int kSmemBytes = kOffBar + 512 + 1024;
+  static constexpr int kOffList = kOffBar + 512;  // block-sparse: the CTA's key-tile list
+  static constexpr int kSmemBytesSparse = kOffList + 4 * kMaxSparseTiles + 1024;
   __device__ static constexpr uint32_t colS(int t) { return static_cast<uint32_t>(t) * 128u; }
   __device__ static constexpr uint32_t colO(int t) { return 256u + static_cast<uint32_t>(t) * D; }
   static constexpr uint32_t kIdescS = idesc_e4m3(kBM, kBN, 0, 0);
@@ -79,6 +81,7 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, unsig
 
 __device__ __forceinline__ bool warp_all(bool ok) { return __all_sync(0xffffffffu, ok); }
 
+template <bool kSparse>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_fp8_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const FwdArgs a, const float out_scale,
@@ -109,7 +112,56 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
   const int kbase = klo[0];
-  const int nk = (nkt[1] > 0) ? max(klo[0] + nkt[0], klo[1] + nkt[1]) - kbase : nkt[0];
+  int nk = (nkt[1] > 0) ? max(klo[0] + nkt[0], klo[1] + nkt[1]) - kbase : nkt[0];
+
+  // Block-sparse (as in the bf16 kernel): the key tiles of the window range
+  // that the mask keeps for at least one of the two query tiles, ascending, as
+  // (tile << 2 | bits) with bit t set when query tile t uses the tile; nkt[t]
+  // becomes query tile t's count and nk the stream length.
+  const uint32_t* klist = reinterpret_cast<const uint32_t*>(smem + C::kOffList);
+  if constexpr (kSparse) {
+    uint32_t* list = reinterpret_cast<uint32_t*>(smem + C::kOffList);
+    __shared__ int s_wcnt[kThreads / 32];
+    __shared__ int s_cnt[3];
+    const uint8_t* mrow0 = a.block_mask + (static_cast<size_t>(a.mask_heads == 1 ? 0 : h) * a.nb + q0[0] / kBM) * a.nb;
+    const uint8_t* mrow1 = mrow0 + a.nb;
+    if (threadIdx.x < 3) s_cnt[threadIdx.x] = 0;
+    __syncthreads();
+    for (int base = 0; base < nk; base += kThreads) {
+      const int c = base + static_cast<int>(threadIdx.x);
+      const int kt = kbase + c;
+      uint32_t f = 0;
+      if (c < nk) {
+        if (kt >= klo[0] && kt < klo[0] + nkt[0] && mrow0[kt]) f |= 1u;
+        if (kt >= klo[1] && kt < klo[1] + nkt[1] && mrow1[kt]) f |= 2u;
+      }
+      const unsigned bal = __ballot_sync(0xffffffffu, f != 0);
+      if (lane == 0) s_wcnt[warp] = __popc(bal);
+      __syncthreads();
+      int off = s_cnt[2];
+      for (int w2 = 0; w2 < warp; ++w2) off += s_wcnt[w2];
+      if (f) {
+        list[off + __popc(bal & ((1u << lane) - 1u))] = (static_cast<uint32_t>(kt) << 2) | f;
+        if (f & 1u) atomicAdd(&s_cnt[0], 1);
+        if (f & 2u) atomicAdd(&s_cnt[1], 1);
+      }
+      __syncthreads();
+      if (threadIdx.x == 0) {
+        int tot = 0;
+        for (int w2 = 0; w2 < kThreads / 32; ++w2) tot += s_wcnt[w2];
+        s_cnt[2] += tot;
+      }
+      __syncthreads();
+    }
+    nkt[0] = s_cnt[0];
+    nkt[1] = s_cnt[1];
+    nk = s_cnt[2];
+  }
+  // key tile of stream position j, and whether query tile t uses it (dense: the window ranges)
+  auto stream_tile = [&](int j) -> int { return kSparse ? static_cast<int>(klist[j] >> 2) : kbase + j; };
+  auto uses = [&](int t, int j) -> bool {
+    return kSparse ? ((klist[j] >> t) & 1u) != 0 : (kbase + j >= klo[t] && kbase + j < klo[t] + nkt[t]);
+  };
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
@@ -151,7 +203,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       float m = -INFINITY;
       float l = 0.f;
       bool ok = true;
+      int e = -1;  // stream position of this tile's j-th key tile
       for (int j = 0; j < nkt[t]; ++j) {
+        if constexpr (kSparse) {
+          do {
+            ++e;
+          } while (!uses(t, e));
+        } else {
+          e = klo[t] - kbase + j;
+        }
         ok = warp_all(wait_bar(&bars->s_full[t], j & 1, w, 8));
         if (!ok) break;
         tc_fence_after();
@@ -162,7 +222,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int c = 0; c < kBN / 32; ++c) reg_fence32(sr + c * 32);
 
-        const int k0 = (klo[t] + j) * kBN;
+        const int k0 = stream_tile(e) * kBN;
         const bool need_mask = (k0 + kBN > a.N) || (k0 + kBN - 1 > q0[t] + a.wr) || (k0 < q0[t] + kBM - 1 - a.wl);
         if (need_mask) {
           const int hi = min(a.N - 1, qrow + a.wr);
@@ -228,6 +288,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(&bars->p_full[t]);
       }
       // ---- epilogue ----
+      if (ok && nkt[t] == 0 && qrow < a.N) {
+        // block-sparse: no key is visible to this row: O = 0, LSE = -inf
+        __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.O) + ((static_cast<size_t>(b) * a.N + qrow) * a.H + h) * D;
+#pragma unroll
+        for (int c = 0; c < D; c += 8) st_global_v4(orow + c, 0u, 0u, 0u, 0u);
+        a.LSE[(static_cast<size_t>(b) * a.H + h) * a.N + qrow] = -INFINITY;
+      }
       if (ok && nkt[t] > 0) {
         ok = warp_all(wait_bar(&bars->o_done[t], (nkt[t] - 1) & 1, w, 9));
         if (ok) {
@@ -276,10 +343,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int n = j / C::kStages;
           if (j >= C::kStages && !wait_bar(&bars->k_empty[s], (n - 1) & 1, w, 1)) break;
           mbar_arrive_expect_tx(&bars->k_full[s], C::kTile);
-          tma_load_4d(smem + C::kOffK + s * C::kTile, &tmK, &bars->k_full[s], 0, (kbase + j) * kBN, hk, b);
+          tma_load_4d(smem + C::kOffK + s * C::kTile, &tmK, &bars->k_full[s], 0, stream_tile(j) * kBN, hk, b);
           if (j >= C::kStages && !wait_bar(&bars->v_empty[s], (n - 1) & 1, w, 2)) break;
           mbar_arrive_expect_tx(&bars->v_full[s], C::kTile);
-          tma_load_4d(smem + C::kOffV + s * C::kTile, &tmV, &bars->v_full[s], 0, (kbase + j) * kBN, hk, b);
+          tma_load_4d(smem + C::kOffV + s * C::kTile, &tmV, &bars->v_full[s], 0, stream_tile(j) * kBN, hk, b);
         }
       }
     } else if (warp == 9) {
@@ -308,15 +375,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                        C::kIdescPV, (acc || kk > 0) ? 1u : 0u);
           umma_commit(&bars->o_done[t]);
         };
-        auto local = [&](int t, int j) { return j - (klo[t] - kbase); };
-        auto active = [&](int t, int j) { return local(t, j) >= 0 && local(t, j) < nkt[t]; };
+        // jl[t]: how many of query tile t's key tiles have had their P V issued
+        int jl[2] = {0, 0};
         // issue order as in the bf16 kernel: S_t(j+1) right behind PV_t(j), which
         // reads P_t(j) from the same columns (the tensor pipe keeps issue order)
-        bool ok = wait_bar(&bars->q_full, 0, w, 3) && wait_bar(&bars->k_full[0], 0, w, 4);
+        bool ok = nk > 0 && wait_bar(&bars->q_full, 0, w, 3) && wait_bar(&bars->k_full[0], 0, w, 4);
         if (ok) {
           tc_fence_after();
           for (int t = 0; t < 2; ++t)
-            if (active(t, 0)) issue_s(t, 0);
+            if (uses(t, 0)) issue_s(t, 0);
           umma_commit(&bars->k_empty[0]);
         }
         for (int j = 0; ok && j < nk; ++j) {
@@ -325,13 +392,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!(ok = wait_bar(&bars->v_full[s], (j / C::kStages) & 1, w, 6))) break;
           bool next_k = false;
           for (int t = 0; t < 2; ++t) {
-            if (active(t, j)) {
-              const int jl = local(t, j);
-              if (!(ok = wait_bar(&bars->p_full[t], jl & 1, w, 7))) break;
+            if (uses(t, j)) {
+              if (!(ok = wait_bar(&bars->p_full[t], jl[t] & 1, w, 7))) break;
               tc_fence_after();
-              issue_pv(t, s, jl > 0);
+              issue_pv(t, s, jl[t] > 0);
+              ++jl[t];
             }
-            if (j + 1 < nk && active(t, j + 1)) {
+            if (j + 1 < nk && uses(t, j + 1)) {
               if (!next_k) {
                 if (!(ok = wait_bar(&bars->k_full[sn], ((j + 1) / C::kStages) & 1, w, 5))) break;
                 tc_fence_after();
@@ -363,11 +430,13 @@ cudaError_t launch_fwd_fp8(const CUtensorMap& tq, const CUtensorMap& tk, const C
                            float out_scale, const DevCtl& c, cudaStream_t s) {
   const int nqb = (a.N + 2 * kBM - 1) / (2 * kBM);
   const dim3 grid(nqb, a.H, a.B);
-  constexpr int smem = Cfg::kSmemBytes;
-  cudaError_t e = cudaFuncSetAttribute(fwd_fp8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e != cudaSuccess) return e;
-  fwd_fp8_kernel<<<grid, kThreads, smem, s>>>(tq, tk, tv, a, out_scale, c);
-  return cudaGetLastError();
+  auto run = [&](auto kernel, int smem) -> cudaError_t {
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    kernel<<<grid, kThreads, smem, s>>>(tq, tk, tv, a, out_scale, c);
+    return cudaGetLastError();
+  };
+  return a.block_mask ? run(fwd_fp8_kernel<true>, Cfg::kSmemBytesSparse) : run(fwd_fp8_kernel<false>, Cfg::kSmemBytes);
 }
 
 }  // namespace fa

@@ -151,6 +151,16 @@ int fa_fwd_fp8(const void* Q, const void* K, const void* V, void* O, float* LSE,
                void* stream);
 
 /*
+ * The 8-bit forward under a block-sparse mask: block_mask and mask_heads as
+ * fa_fwd_blocksparse (NULL: no mask, which is fa_fwd_fp8), the other arguments
+ * as fa_fwd_fp8.  Key blocks a query block does not see are neither loaded nor
+ * multiplied; a row that sees no key gets O = 0 and LSE = -inf.
+ */
+int fa_fwd_fp8_blocksparse(const void* Q, const void* K, const void* V, void* O, float* LSE, int B, int H, int Hkv,
+                           int N, int d, float scale, float scale_q, float scale_k, float scale_v, int window_left,
+                           int window_right, const void* block_mask, int mask_heads, void* stream);
+
+/*
  * Bytes of device workspace fa_bwd needs for this problem: an fp32 dQ
  * accumulator [B, N, H, d] plus two fp32 [B, H, roundup(N, 128)] rows
  * (rowsum(dO * O) and LSE * log2 e), each region 256-byte aligned.  This is

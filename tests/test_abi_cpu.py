@@ -288,3 +288,15 @@ def test_header_is_plain_c_and_links(L, tmp_path):
                     "-L", str(lib_dir), "-lfa", f"-Wl,-rpath,{lib_dir}"], check=True)
     out = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()
     assert out[0] == str(L.fa_version())
+
+
+def test_fp8_blocksparse_validation(L):
+    """fa_fwd_fp8_blocksparse: mask_heads must be 1 or H; valid arguments reach the
+    alignment check; a null mask is the plain 8-bit forward."""
+    f = L.fa_fwd_fp8_blocksparse
+    ok = (0.1, 1.0, 1.0, 1.0)
+    assert f(16, 16, 16, 16, 16, 1, 4, 2, 256, 128, *ok, -1, -1, 16, 3, None) == -1
+    assert f(16, 16, 16, 16, 16, 1, 4, 2, 256, 64, *ok, -1, -1, 16, 1, None) == -2
+    assert f(16, 16, 16, 16, 16, 1, 4, 2, 4096 * 128 + 128, 128, *ok, -1, -1, 16, 1, None) == -8
+    assert f(8, 16, 16, 16, 16, 1, 4, 2, 256, 128, *ok, -1, -1, 16, 4, None) == -3
+    assert f(8, 16, 16, 16, 16, 1, 4, 2, 256, 128, *ok, -1, -1, None, 0, None) == -3

@@ -47,12 +47,12 @@ def _fp8_inputs(B, N, H, Hkv, seed, spike_frac=0.0):
     return (cq, ck, cv), (sq, sk, sv), deq
 
 
-def _bound(qd, kd, vd, scale, causal, window, rows=None):
+def _bound(qd, kd, vd, scale, causal, window, rows=None, block_mask=None):
     """Per-element error bound of the e4m3 probabilities (see the module docstring), one head."""
     if rows is None:
         rows = np.arange(qd.shape[0])
     s = oracle.scores_head(qd[rows], kd, scale, False)
-    hidden = oracle.hidden_keys(rows, kd.shape[0], causal, window)
+    hidden = oracle.hidden_keys(rows, kd.shape[0], causal, window, block_mask)
     s = np.where(hidden, -np.inf, s)
     p, _ = oracle.probs_head(s)
     av = np.abs(vd)
@@ -115,3 +115,34 @@ def test_fp8_refuses_other_head_dims():
     x = torch.zeros(1, 128, 1, 64, dtype=torch.float8_e4m3fn, device="cuda")
     with pytest.raises(fa.FAError):
         fa.fwd_fp8(x, x, x, 1.0, 1.0, 1.0)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("n,H,Hkv,heads_mask", [(384, 2, 2, 1), (700, 4, 2, 4), (1000, 2, 1, 1)])
+def test_fp8_blocksparse(n, H, Hkv, heads_mask):
+    """The 8-bit forward under a 0/1 mask over 128 x 128 blocks (one shared or one
+    per query head, with an empty block row): every element within the e4m3
+    bound of the oracle on the dequantised inputs; empty rows O = 0, LSE = -inf."""
+    need_gpu()
+    nb = (n + 127) // 128
+    m = (np.random.default_rng(n + H).random((heads_mask, nb, nb)) < 0.5).astype(np.uint8)
+    m[:, nb // 2, :] = 0
+    mask = m[0] if heads_mask == 1 else m
+    (cq, ck, cv), (sq, sk, sv), (dq, dk, dv) = _fp8_inputs(1, n, H, Hkv, seed=n)
+    scale = float(np.float32(1.0 / math.sqrt(128)))
+    o, lse = fa.fwd_fp8(cq.cuda(), ck.cuda(), cv.cuda(), sq, sk, sv, scale=scale,
+                        block_mask=torch.from_numpy(mask).cuda())
+    torch.cuda.synchronize()
+    assert fa.last_device_status()[0] == 0
+    o, lse = f64(o), f64(lse)
+    G = H // Hkv
+    for h in range(H):
+        mh = mask if heads_mask == 1 else mask[h]
+        qh, kh, vh = dq[0, :, h].numpy(), dk[0, :, h // G].numpy(), dv[0, :, h // G].numpy()
+        rows = np.arange(n)
+        ro, rl = oracle.forward_rows_head(qh, kh, vh, rows, scale, False, block_mask=mh)
+        bound = _bound(qh, kh, vh, scale, False, None, rows=rows, block_mask=mh)
+        assert (np.abs(o[0, :, h] - ro) <= bound).all(), h
+        both_inf = np.isneginf(lse[0, h]) & np.isneginf(rl)
+        with np.errstate(invalid="ignore"):
+            assert np.all(both_inf | (np.abs(lse[0, h] - rl) <= TOL_LSE)), h
