@@ -33,12 +33,16 @@ _LIB = None
 
 # Every symbol include/fa.h declares.
 EXPORTED = ("fa_fwd", "fa_bwd_workspace_size", "fa_bwd", "fa_status_string", "fa_last_cuda_error",
-            "fa_last_device_status", "fa_set_wait_limit_ms", "fa_debug_inject", "fa_debug_umma",
+            "fa_last_device_status", "fa_set_wait_limit_ms",
             "fa_version", "fa_set_kernel_events", "fa_bwd_static_scratch", "fa_fwd_gqa", "fa_bwd_gqa",
-            "fa_fwd_window", "fa_bwd_window", "fa_debug_umma_f8", "fa_fwd_fp8",
+            "fa_fwd_window", "fa_bwd_window", "fa_fwd_fp8",
             "fa_fwd_blocksparse", "fa_bwd_blocksparse", "fa_merge_partial", "fa_accumulate_bf16",
             "fa_cast_bf16", "fa_bwd_workspace_size_gqa", "fa_decode_paged", "fa_decode_workspace_size",
             "fa_fwd_fp8_blocksparse")
+# Test-only symbols (csrc/fa_testing.h): the first in libfa.so, the others in the
+# separate test library libfa_probe.so.
+TESTING_EXPORTED = {"libfa.so": ("fa_debug_inject",), "libfa_probe.so": ("fa_debug_umma", "fa_debug_umma_f8")}
+_PROBE = None
 
 
 class FAError(RuntimeError):
@@ -110,10 +114,6 @@ def lib() -> ctypes.CDLL:
     L.fa_set_wait_limit_ms.restype = None
     L.fa_debug_inject.argtypes = [i]
     L.fa_debug_inject.restype = None
-    L.fa_debug_umma.argtypes = [vp, vp, vp, i, i, i, i, i, vp]
-    L.fa_debug_umma.restype = i
-    L.fa_debug_umma_f8.argtypes = [vp, vp, vp, i, i, i, vp]
-    L.fa_debug_umma_f8.restype = i
     L.fa_bwd_static_scratch.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, i, vp]
     L.fa_bwd_static_scratch.restype = i
     L.fa_set_kernel_events.argtypes = [vp, vp]
@@ -122,6 +122,24 @@ def lib() -> ctypes.CDLL:
     L.fa_version.restype = i
     _LIB = L
     return L
+
+
+def probe_lib() -> ctypes.CDLL:
+    """Load the test library ``libfa_probe.so`` (single MMA tile probes, test-only)."""
+    global _PROBE
+    if _PROBE is not None:
+        return _PROBE
+    path = _PKG / "libfa_probe.so"
+    if not path.exists():
+        raise FAError(-6, f"{path} is missing; build it with `python -m exact_io_aware_51_b200.build`")
+    P = ctypes.CDLL(str(path))
+    vp, i = ctypes.c_void_p, ctypes.c_int
+    P.fa_debug_umma.argtypes = [vp, vp, vp, i, i, i, i, i, vp]
+    P.fa_debug_umma.restype = i
+    P.fa_debug_umma_f8.argtypes = [vp, vp, vp, i, i, i, vp]
+    P.fa_debug_umma_f8.restype = i
+    _PROBE = P
+    return P
 
 
 def status_string(status: int) -> str:
@@ -407,7 +425,7 @@ def debug_umma(a: torch.Tensor, b: torch.Tensor, a_mn_major: int, b_mn_major: in
     """One tcgen05 MMA tile D = A B^T (test-only): a [128, K], b [N, K] bf16 cuda."""
     n, kdim = b.shape
     dmat = torch.empty((128, n), dtype=torch.float32, device=a.device)
-    rc = lib().fa_debug_umma(a.data_ptr(), b.data_ptr(), dmat.data_ptr(), n, kdim, int(a_mn_major),
+    rc = probe_lib().fa_debug_umma(a.data_ptr(), b.data_ptr(), dmat.data_ptr(), n, kdim, int(a_mn_major),
                              int(b_mn_major), int(a_tmem), _stream_handle(stream, a.device))
     if rc != 0:
         raise FAError(rc, "fa_debug_umma")
@@ -418,7 +436,7 @@ def debug_umma_f8(a: torch.Tensor, b: torch.Tensor, b_mn_major: int, a_tmem: int
     """One 8-bit tcgen05 MMA tile D = A B^T (test-only): a [128, 128], b [N, 128] e4m3 (uint8 bytes) cuda."""
     n = b.shape[0]
     dmat = torch.empty((128, n), dtype=torch.float32, device=a.device)
-    rc = lib().fa_debug_umma_f8(a.data_ptr(), b.data_ptr(), dmat.data_ptr(), n, int(b_mn_major), int(a_tmem),
+    rc = probe_lib().fa_debug_umma_f8(a.data_ptr(), b.data_ptr(), dmat.data_ptr(), n, int(b_mn_major), int(a_tmem),
                                 _stream_handle(stream, a.device))
     if rc != 0:
         raise FAError(rc, "fa_debug_umma_f8")

@@ -1,9 +1,11 @@
 """Build the CUDA library ``libfa.so`` in-tree (sm_100a only).
 
 ``python -m exact_io_aware_51_b200.build`` compiles every ``csrc/*.cu`` with
-nvcc for ``sm_100a`` into ``exact_io_aware_51_b200/libfa.so``.  nvcc
-cross-compiles without a GPU.  The CUDA runtime is linked statically, so the
-library only needs the driver at run time.
+nvcc for ``sm_100a``: the product library ``exact_io_aware_51_b200/libfa.so``
+and, from ``fa_probe.cu`` alone, the test library ``libfa_probe.so`` (single
+MMA tile probes; declared in ``csrc/fa_testing.h``, not in the public header).
+nvcc cross-compiles without a GPU.  The CUDA runtime is linked statically, so
+the libraries only need the driver at run time.
 """
 
 from __future__ import annotations
@@ -21,9 +23,11 @@ CSRC = PKG / "csrc"
 INCLUDE = ROOT / "include"
 BUILD = PKG / "_build"
 LIB = PKG / "libfa.so"
-SOURCES = ("fa_api.cu", "fa_fwd_bf16.cu", "fa_fwd_fp8.cu", "fa_fwd_f32.cu", "fa_bwd.cu", "fa_probe.cu",
+SOURCES = ("fa_api.cu", "fa_fwd_bf16.cu", "fa_fwd_fp8.cu", "fa_fwd_f32.cu", "fa_bwd.cu",
            "fa_bwd_static.cu", "fa_ring.cu",
            "fa_bwd64.cu", "fa_decode.cu")
+PROBE_SOURCES = ("fa_probe.cu",)
+PROBE_LIB = PKG / "libfa_probe.so"
 ARCH = ("-gencode", "arch=compute_100a,code=sm_100a")
 FLAGS = ("-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall",
          "--expt-relaxed-constexpr")
@@ -37,19 +41,20 @@ def nvcc() -> str:
 
 
 def _deps():
-    return [CSRC / s for s in SOURCES] + list(CSRC.glob("*.cuh")) + list(CSRC.glob("*.h")) + [INCLUDE / "fa.h", pathlib.Path(__file__)]
+    return ([CSRC / s for s in SOURCES + PROBE_SOURCES] + list(CSRC.glob("*.cuh")) + list(CSRC.glob("*.h"))
+            + [INCLUDE / "fa.h", pathlib.Path(__file__)])
 
 
 def up_to_date() -> bool:
-    if not LIB.exists():
+    if not LIB.exists() or not PROBE_LIB.exists():
         return False
-    t = LIB.stat().st_mtime
+    t = min(LIB.stat().st_mtime, PROBE_LIB.stat().st_mtime)
     return all(p.stat().st_mtime <= t for p in _deps())
 
 
 def _compile(src: pathlib.Path, verbose: bool) -> pathlib.Path:
     obj = BUILD / (src.stem + ".o")
-    cmd = [nvcc(), *ARCH, *FLAGS, "-I", str(INCLUDE), "-c", str(src), "-o", str(obj)]
+    cmd = [nvcc(), *ARCH, *FLAGS, "-I", str(INCLUDE), "-I", str(CSRC), "-c", str(src), "-o", str(obj)]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
         print(" ".join(cmd), flush=True)
@@ -66,14 +71,16 @@ def build(force: bool = False, verbose: bool = False) -> pathlib.Path:
     if not force and up_to_date():
         return LIB
     BUILD.mkdir(exist_ok=True)
-    with concurrent.futures.ThreadPoolExecutor(max_workers=len(SOURCES)) as ex:
-        objs = list(ex.map(lambda s: _compile(CSRC / s, verbose), SOURCES))
-    tmp = LIB.with_suffix(".so.tmp")
-    cmd = [nvcc(), *ARCH, "-shared", "-o", str(tmp), *map(str, objs), "-cudart", "static"]
-    r = subprocess.run(cmd, capture_output=True, text=True)
-    if r.returncode != 0:
-        raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
-    os.replace(tmp, LIB)
+    every = SOURCES + PROBE_SOURCES
+    with concurrent.futures.ThreadPoolExecutor(max_workers=len(every)) as ex:
+        objs = dict(zip(every, ex.map(lambda s: _compile(CSRC / s, verbose), every)))
+    for lib, srcs in ((LIB, SOURCES), (PROBE_LIB, PROBE_SOURCES)):
+        tmp = lib.with_suffix(".so.tmp")
+        cmd = [nvcc(), *ARCH, "-shared", "-o", str(tmp), *(str(objs[s]) for s in srcs), "-cudart", "static"]
+        r = subprocess.run(cmd, capture_output=True, text=True)
+        if r.returncode != 0:
+            raise RuntimeError(f"link of {lib.name} failed:\n{r.stdout}\n{r.stderr}")
+        os.replace(tmp, lib)
     return LIB
 
 

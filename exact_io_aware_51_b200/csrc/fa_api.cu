@@ -13,6 +13,7 @@
 
 #include "fa.h"
 #include "fa_internal.h"
+#include "fa_testing.h"
 
 namespace fa {
 
@@ -676,31 +677,6 @@ int fa_cast_bf16(void* out, const float* in, long long n, void* stream) {
   int rc = device_state(&st);
   if (rc) return rc;
   cudaError_t e = launch_cast(out, in, n, static_cast<cudaStream_t>(stream));
-  if (e != cudaSuccess) return fail_cuda(e);
-  return FA_OK;
-}
-
-int fa_debug_umma(const void* A, const void* B, float* D, int N, int K, int a_mn_major, int b_mn_major, int a_tmem,
-                  void* stream) {
-  if (!A || !B || !D) return FA_ERR_INVALID_ARG;
-  if ((N != 64 && N != 128) || (K != 64 && K != 128)) return FA_ERR_UNSUPPORTED;
-  DeviceState* st = nullptr;
-  int rc = device_state(&st);
-  if (rc) return rc;
-  cudaError_t e = launch_umma_probe(A, B, D, N, K, a_mn_major ? 1 : 0, b_mn_major ? 1 : 0, a_tmem ? 1 : 0,
-                                    static_cast<cudaStream_t>(stream));
-  if (e != cudaSuccess) return fail_cuda(e);
-  return FA_OK;
-}
-
-int fa_debug_umma_f8(const void* A, const void* B, float* D, int N, int b_mn_major, int a_tmem, void* stream) {
-  if (!A || !B || !D) return FA_ERR_INVALID_ARG;
-  if (N != 64 && N != 128) return FA_ERR_UNSUPPORTED;
-  DeviceState* st = nullptr;
-  int rc = device_state(&st);
-  if (rc) return rc;
-  cudaError_t e =
-      launch_umma_probe_f8(A, B, D, N, b_mn_major ? 1 : 0, a_tmem ? 1 : 0, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return fail_cuda(e);
   return FA_OK;
 }

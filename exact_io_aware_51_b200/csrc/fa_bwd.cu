@@ -166,13 +166,6 @@ struct BwdBars {
 static_assert(sizeof(BwdBars) <= 256, "barrier block");
 static_assert(BwdCfg::kOffDQS % 1024 == 0 && BwdCfg::kSmemBytes <= 232448, "shared memory layout");
 
-__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, unsigned long long limit_ns) {
-  const uint64_t t0 = globaltimer_ns();
-  while (!mbar_try_wait(bar, parity)) {
-    if (globaltimer_ns() - t0 > limit_ns) break;
-  }
-}
-
 __device__ __forceinline__ bool warp_all(bool ok) { return __all_sync(0xffffffffu, ok); }
 
 // TMA reduce-add of a shared-memory tile into global memory (fp32), and the
@@ -567,6 +560,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         }
+        int q_issued = 0;
         for (int i = 0; i < nq; ++i) {
           const int st = i % kStages;
           const int n = i / kStages;
@@ -590,7 +584,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           bulk_load(smem + C::kOffL + st * 512, a.LSE2 + bh * a.Npad + q0, 512, &bars->q_full[st]);
           bulk_load(smem + C::kOffDv + st * 512, a.Dvec + bh * a.Npad + q0, 512, &bars->q_full[st]);
+          ++q_issued;
         }
+        // teardown: no copy of this CTA may still be writing its shared memory
+        drain_wait(&bars->kv_full, 0, ctl.limit_ns);
+        drain_ring(bars->q_full, kStages, q_issued, ctl.limit_ns);
       }
     } else if (bars->abort == 0 && warp == 13) {
       // ===================== MMA issuer =====================

@@ -12,8 +12,11 @@
 // Cost and limits:
 //   * the array is kStaticScratchBytes (64 MiB) of device memory on every GPU
 //     that loads the library, held until the process exits;
-//   * problems whose workspace (fa_bwd_workspace_size) exceeds it are refused
-//     with FA_ERR_TOO_LARGE;
+//   * problems whose base workspace (the fp32 dQ accumulator and the two
+//     per-row arrays) exceeds it are refused with FA_ERR_TOO_LARGE; a problem
+//     whose base fits but whose split-walk dK / dV accumulators do not (so
+//     fa_bwd_workspace_size is larger than the array) runs with unsplit walks,
+//     which gives the same gradients, only without the small-grid speed-up;
 //   * every call shares the array and leaves its contents behind; the
 //     backward's preprocess kernel rewrites everything the later kernels read
 //     (it zeroes the dQ accumulator and fills both per-row arrays), so nothing
@@ -41,27 +44,25 @@ constexpr int kMaxScratchDevices = 64;
 static __device__ __align__(256) unsigned char g_bwd_scratch[kStaticScratchBytes];
 
 struct ScratchSlot {
-  std::once_flag once;
+  std::mutex mu;
   void* ptr = nullptr;
-  cudaError_t err = cudaSuccess;
 };
 ScratchSlot g_slots[kMaxScratchDevices];
 
-// Device address of the scratch array on the current device (looked up once
-// per device, with that device current).
+// Device address of the scratch array on the current device, looked up with
+// that device current.  Only a successful lookup is kept; after a failure the
+// next call tries again.
 int scratch_address(void** out) {
   int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return FA_ERR_LAUNCH;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_LAUNCH;
   if (dev < 0 || dev >= kMaxScratchDevices) return FA_ERR_ARCH;
   ScratchSlot& s = g_slots[dev];
-  std::call_once(s.once, [&] {
-    e = cudaSetDevice(dev);
-    if (e == cudaSuccess) e = cudaGetSymbolAddress(&s.ptr, g_bwd_scratch);
-    s.err = e;
-    if (e != cudaSuccess) s.ptr = nullptr;
-  });
-  if (s.err != cudaSuccess || s.ptr == nullptr) return FA_ERR_LAUNCH;
+  std::lock_guard<std::mutex> lock(s.mu);
+  if (s.ptr == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_bwd_scratch) != cudaSuccess || p == nullptr) return FA_ERR_LAUNCH;
+    s.ptr = p;
+  }
   *out = s.ptr;
   return FA_OK;
 }

@@ -160,6 +160,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
       const int R = min(P, kTileKeys);  // rows per box (the maps' box height)
+      int issued = 0;
       for (int t = 0; t < ntiles; ++t) {
         const int st = t % C::kStages;
         if (t >= C::kStages && !wait_bar(&bars->empty[st], ((t / C::kStages) - 1) & 1, w, 0xC1)) break;
@@ -178,7 +179,10 @@ __global__ void __launch_bounds__(kThreads, 2)
             tma_load_2d(vs + hf * kHalfBytes + bx * R * 128, &tmV, &bars->full[st], hkv * D + hf * 64, row);
           }
         }
+        ++issued;
       }
+      // no copy of this CTA may still be writing its shared memory when it exits
+      drain_ring(bars->full, C::kStages, issued, ctl.limit_ns);
     }
     return;  // the consumers' merge below syncs only the four consumer warps
   }

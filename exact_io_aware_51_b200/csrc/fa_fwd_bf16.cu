@@ -93,15 +93,6 @@ struct FwdBars {
   int abort;
 };
 
-// Wait on a barrier ignoring the CTA abort flag (used only to drain in-flight
-// MMAs before TMEM is released); still bounded.
-__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, unsigned long long limit_ns) {
-  const uint64_t t0 = globaltimer_ns();
-  while (!mbar_try_wait(bar, parity)) {
-    if (globaltimer_ns() - t0 > limit_ns) break;
-  }
-}
-
 __device__ __forceinline__ bool warp_all(bool ok) { return __all_sync(0xffffffffu, ok); }
 
 template <int D, bool kSparse>
@@ -375,6 +366,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_load_4d(smem + C::kOffQ + t * C::kTileBytes + c * C::kSubBytes, &tmQ, &bars->q_full, c * 64,
                         q0[t], h, b);
         }
+        int k_issued = 0, v_issued = 0;
         for (int j = 0; j < nk; ++j) {
           const int s = j % C::kStages;
           const int n = j / C::kStages;
@@ -384,12 +376,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int c = 0; c < C::kSub; ++c)
             tma_load_4d(smem + C::kOffK + s * C::kTileBytes + c * C::kSubBytes, &tmK, &bars->k_full[s], c * 64,
                         stream_tile(j) * kBN, hk, b);
+          ++k_issued;
           if (j >= C::kStages && !wait_bar(&bars->v_empty[s], (n - 1) & 1, w, 2)) break;
           mbar_arrive_expect_tx(&bars->v_full[s], C::kTileBytes);
           for (int c = 0; c < C::kSub; ++c)
             tma_load_4d(smem + C::kOffV + s * C::kTileBytes + c * C::kSubBytes, &tmV, &bars->v_full[s], c * 64,
                         stream_tile(j) * kBN, hk, b);
+          ++v_issued;
         }
+        // teardown: no copy of this CTA may still be writing its shared memory
+        drain_wait(&bars->q_full, 0, ctl.limit_ns);
+        drain_ring(bars->k_full, C::kStages, k_issued, ctl.limit_ns);
+        drain_ring(bars->v_full, C::kStages, v_issued, ctl.limit_ns);
       }
     } else if (warp == 9) {
       // ===================== MMA issuer (one thread) =====================

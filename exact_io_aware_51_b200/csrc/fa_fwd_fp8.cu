@@ -72,13 +72,6 @@ struct Bars {
   int abort;
 };
 
-__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, unsigned long long limit_ns) {
-  const uint64_t t0 = globaltimer_ns();
-  while (!mbar_try_wait(bar, parity)) {
-    if (globaltimer_ns() - t0 > limit_ns) break;
-  }
-}
-
 __device__ __forceinline__ bool warp_all(bool ok) { return __all_sync(0xffffffffu, ok); }
 
 template <bool kSparse>
@@ -338,16 +331,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive_expect_tx(&bars->q_full, qbytes);
         for (int t = 0; t < 2; ++t)
           if (nkt[t] > 0) tma_load_4d(smem + C::kOffQ + t * C::kTile, &tmQ, &bars->q_full, 0, q0[t], h, b);
+        int k_issued = 0, v_issued = 0;
         for (int j = 0; j < nk; ++j) {
           const int s = j % C::kStages;
           const int n = j / C::kStages;
           if (j >= C::kStages && !wait_bar(&bars->k_empty[s], (n - 1) & 1, w, 1)) break;
           mbar_arrive_expect_tx(&bars->k_full[s], C::kTile);
           tma_load_4d(smem + C::kOffK + s * C::kTile, &tmK, &bars->k_full[s], 0, stream_tile(j) * kBN, hk, b);
+          ++k_issued;
           if (j >= C::kStages && !wait_bar(&bars->v_empty[s], (n - 1) & 1, w, 2)) break;
           mbar_arrive_expect_tx(&bars->v_full[s], C::kTile);
           tma_load_4d(smem + C::kOffV + s * C::kTile, &tmV, &bars->v_full[s], 0, stream_tile(j) * kBN, hk, b);
+          ++v_issued;
         }
+        // teardown: no copy of this CTA may still be writing its shared memory
+        drain_wait(&bars->q_full, 0, ctl.limit_ns);
+        drain_ring(bars->k_full, C::kStages, k_issued, ctl.limit_ns);
+        drain_ring(bars->v_full, C::kStages, v_issued, ctl.limit_ns);
       }
     } else if (warp == 9) {
       // ===================== MMA issuer (one thread) =====================

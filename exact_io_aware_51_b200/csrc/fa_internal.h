@@ -144,10 +144,4 @@ cudaError_t launch_merge(float* o_acc, float* lse_acc, const void* o_part, const
 cudaError_t launch_accumulate(float* acc, const void* part, long long n, int init, cudaStream_t s);
 cudaError_t launch_cast(void* out, const float* in, long long n, cudaStream_t s);
 
-// Test-only single-tile MMA probe (see fa_debug_umma in the public header).
-cudaError_t launch_umma_probe(const void* A, const void* B, float* D, int N, int K, int a_mn_major,
-                              int b_mn_major, int a_tmem, cudaStream_t s);
-cudaError_t launch_umma_probe_f8(const void* A, const void* B, float* D, int N, int b_mn_major, int a_tmem,
-                                 cudaStream_t s);
-
 }  // namespace fa

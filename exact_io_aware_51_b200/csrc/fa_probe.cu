@@ -5,9 +5,14 @@
 // and A read from tensor memory.  The threads place A and B in shared memory
 // with the same swizzle the TMA produces, one thread issues the MMAs, and the
 // fp32 result is read back through tcgen05.ld.
+//
+// It is built into its own test library (libfa_probe.so), outside the product
+// library, and declared in fa_testing.h, not in the public header.
 #include <cuda_bf16.h>
+#include <cuda_runtime.h>
 
-#include "fa_internal.h"
+#include "fa.h"
+#include "fa_testing.h"
 #include "sm100.cuh"
 
 namespace fa {
@@ -208,8 +213,6 @@ __global__ void __launch_bounds__(128, 1)
   }
 }
 
-}  // namespace
-
 cudaError_t launch_umma_probe_f8(const void* A, const void* B, float* D, int N, int b_mn, int a_tmem,
                                  cudaStream_t s) {
   constexpr int smem = 32768 + 1024;
@@ -230,4 +233,40 @@ cudaError_t launch_umma_probe(const void* A, const void* B, float* D, int N, int
   return cudaGetLastError();
 }
 
+// The current device must be an sm_100 part (tcgen05).
+int probe_device_ok() {
+  int dev = 0, major = 0, minor = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_LAUNCH;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+    return FA_ERR_LAUNCH;
+  return (major == 10 && minor == 0) ? FA_OK : FA_ERR_ARCH;
+}
+
+}  // namespace
 }  // namespace fa
+
+extern "C" {
+
+int fa_debug_umma(const void* A, const void* B, float* D, int N, int K, int a_mn_major, int b_mn_major, int a_tmem,
+                  void* stream) {
+  if (!A || !B || !D) return FA_ERR_INVALID_ARG;
+  if ((N != 64 && N != 128) || (K != 64 && K != 128)) return FA_ERR_UNSUPPORTED;
+  const int rc = fa::probe_device_ok();
+  if (rc != FA_OK) return rc;
+  const cudaError_t e = fa::launch_umma_probe(A, B, D, N, K, a_mn_major ? 1 : 0, b_mn_major ? 1 : 0, a_tmem ? 1 : 0,
+                                              static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
+}
+
+int fa_debug_umma_f8(const void* A, const void* B, float* D, int N, int b_mn_major, int a_tmem, void* stream) {
+  if (!A || !B || !D) return FA_ERR_INVALID_ARG;
+  if (N != 64 && N != 128) return FA_ERR_UNSUPPORTED;
+  const int rc = fa::probe_device_ok();
+  if (rc != FA_OK) return rc;
+  const cudaError_t e =
+      fa::launch_umma_probe_f8(A, B, D, N, b_mn_major ? 1 : 0, a_tmem ? 1 : 0, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
+}
+
+}  // extern "C"

@@ -8,7 +8,7 @@ Remez exchange algorithm.  The kernel rounds P to bf16 (relative step 2^-8),
 so a relative error near 1e-4 is far below what the result can show.
 
 Run `python gen_exp2_poly.py` to print the coefficients and the error bound;
-the printed values are the ones in fa_fwd_bf16.cu.
+the printed values are the ones exp2_poly2 in sm100.cuh uses.
 """
 
 import numpy as np

@@ -115,6 +115,28 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, const W
   return wait_slow(bar, parity, w, site);
 }
 
+// Teardown wait: ignores the abort flag but is still bounded.  The MMA thread
+// uses it for its in-flight MMAs before TMEM is released, and the loaders for
+// the bulk copies they issued, so that no CTA exits (and hands its shared
+// memory to the next CTA) while a copy still writes there.
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, unsigned long long limit_ns) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > limit_ns) break;
+  }
+}
+
+// A loader that armed `issued` loads round-robin on the full barriers
+// full[0 .. stages) waits for the last one of each stage.  A phase that the
+// consumers already saw complete passes at once (no later load was armed on
+// that stage, so the barrier is exactly one phase past it).
+__device__ __forceinline__ void drain_ring(uint64_t* full, int stages, int issued, unsigned long long limit_ns) {
+  for (int s = 0; s < stages && s < issued; ++s) {
+    const int last = s + ((issued - 1 - s) / stages) * stages;
+    drain_wait(&full[s], static_cast<uint32_t>(last / stages) & 1u, limit_ns);
+  }
+}
+
 // --------------------------------------------------------------------------
 // TMA (no cluster multicast anywhere in this library)
 // --------------------------------------------------------------------------

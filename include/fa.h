@@ -240,8 +240,11 @@ int fa_bwd_blocksparse(const void* Q, const void* K, const void* V, const void* 
  *   Same arguments and results as fa_bwd, minus the workspace: the scratch is
  *   a 64 MiB array compiled into the library, which every GPU that loads the
  *   library holds until the process exits.  The call allocates nothing.
- *   A problem whose fa_bwd_workspace_size() exceeds 64 MiB is refused with
- *   FA_ERR_TOO_LARGE.
+ *   A problem whose base workspace (the fp32 dQ accumulator and the two
+ *   per-row arrays, i.e. fa_bwd_workspace_size() without the split-walk dK /
+ *   dV accumulators) exceeds 64 MiB is refused with FA_ERR_TOO_LARGE.  When
+ *   the base fits but the split-walk accumulators do not, the walks run
+ *   unsplit: the same gradients, without the small-grid speed-up.
  *   All calls share that one array.  Each call's first kernel rewrites what
  *   the later ones read, so results never depend on an earlier call, but
  *   calls whose kernels overlap on the GPU (other streams, or other host
@@ -351,15 +354,11 @@ int fa_last_cuda_error(void);
 int fa_last_device_status(void* stream, int* detail);
 
 /*
- * Test and diagnostics knobs (process-wide).
- *   fa_set_wait_limit_ms: limit for any single wait inside a kernel
- *     (default 2000 ms, or the FA_TIMEOUT_MS environment variable).
- *   fa_debug_inject: 1 makes the next forward launches' first key-tile
- *     barrier expect 16 bytes that never arrive, so its waits expire and the
- *     launch reports FA_ERR_DEVICE_TIMEOUT; 0 turns it off.
+ * Diagnostics knob (process-wide): the limit for any single wait inside a
+ * kernel (default 2000 ms, or the FA_TIMEOUT_MS environment variable); after
+ * it the launch gives up and reports FA_ERR_DEVICE_TIMEOUT.
  */
 void fa_set_wait_limit_ms(int ms);
-void fa_debug_inject(int mode);
 
 /*
  * Diagnostics: while set, each fa_fwd / fa_bwd call made on this host thread
@@ -369,26 +368,6 @@ void fa_debug_inject(int mode);
  * Pass NULL, NULL to turn it off.  The events stay owned by the caller.
  */
 void fa_set_kernel_events(void* start, void* stop);
-
-/*
- * Test-only: one 128 x N x K tcgen05 MMA tile, D = A B^T, with A [128][K] and
- * B [N][K] bf16 row-major device arrays and D [128][N] fp32.  a_mn_major /
- * b_mn_major choose how the operand is laid out in shared memory (0: the
- * reduction dimension contiguous, 1: the M or N dimension contiguous); a_tmem
- * reads A from tensor memory instead.  N and K must be 64 or 128.  Synchronous
- * on `stream` is not implied.
- */
-int fa_debug_umma(const void* A, const void* B, float* D, int N, int K, int a_mn_major, int b_mn_major,
-                  int a_tmem, void* stream);
-
-/*
- * Test-only: the same probe for the 8-bit MMA (kind::f8f6f4, e4m3 operands,
- * fp32 accumulation) with K = 128: A [128][128] and B [N][128] e4m3 bytes
- * (row-major device arrays), D [128][N] fp32.  b_mn_major stores B with N
- * contiguous; a_tmem reads A from tensor memory (four elements per column).
- * N must be 64 or 128.
- */
-int fa_debug_umma_f8(const void* A, const void* B, float* D, int N, int b_mn_major, int a_tmem, void* stream);
 
 /* Library version: major * 10000 + minor * 100 + patch. */
 int fa_version(void);

@@ -45,6 +45,25 @@ def test_library_exports_every_declared_symbol(L):
         assert getattr(L, name) is not None
 
 
+def test_test_only_symbols_live_outside_the_public_header(L):
+    """fa_debug_* are declared in csrc/fa_testing.h (not include/fa.h) and exported
+    by the library that the binding names for each."""
+    testing = ROOT / "exact_io_aware_51_b200" / "csrc" / "fa_testing.h"
+    text = re.sub(r"/\*.*?\*/", "", testing.read_text(), flags=re.S)
+    declared = sorted(set(re.findall(r"\b(fa_[a-z0-9_]+)\s*\(", text)))
+    listed = sorted(n for names in fa.TESTING_EXPORTED.values() for n in names)
+    assert declared == listed
+    assert not set(declared) & set(declared_functions())
+    for lib_name, names in fa.TESTING_EXPORTED.items():
+        out = subprocess.run(["nm", "-D", "--defined-only", str(fa.lib_path().parent / lib_name)],
+                             capture_output=True, text=True, check=True).stdout
+        exported = set(re.findall(r" T (fa_[a-z0-9_]+)$", out, flags=re.M))
+        for name in names:
+            assert name in exported, (lib_name, name)
+    probe = fa.probe_lib()
+    assert probe.fa_debug_umma(None, None, None, 64, 64, 0, 0, 0, None) == -1
+
+
 def test_status_strings(L):
     for code in (0, -1, -2, -3, -4, -5, -6, -7, -8, -9):
         assert fa.status_string(code) and "unknown" not in fa.status_string(code)

@@ -74,15 +74,15 @@ def test_reference_arm_on_a_non_zero_rank_exits_quietly():
     assert r.stdout.strip() == ""
 
 
-def test_peak_follows_the_power_state_of_the_timed_steps():
-    """Kernels timed while the power cap is active are compared with the sustained
-    GEMM figure; otherwise with the burst one."""
+def test_clock_scaled_fraction():
+    """The fraction at the maximum SM clock is frac x max MHz / median MHz, and
+    None when there is no clock record."""
     sys.path.insert(0, ROOT)
     import bench
-    assert bench.choose_peak({"reasons": ["sw_power_cap"]}, 1660.9, 1397.6)[0] == 1397.6
-    assert bench.choose_peak({"reasons": []}, 1660.9, 1397.6)[0] == 1660.9
-    assert bench.choose_peak({"reasons": None}, 1660.9, 1397.6)[0] == 1660.9
-    assert bench.choose_peak({}, 1660.9, 1397.6)[0] == 1660.9
+    assert abs(bench.clock_scaled(0.6, {"sm_mhz": 1700.0, "sm_max_mhz": 1965.0}) - 0.6 * 1965 / 1700) < 1e-12
+    assert bench.clock_scaled(0.6, {"sm_mhz": None, "sm_max_mhz": 1965.0}) is None
+    assert bench.clock_scaled(0.6, {}) is None
+    assert bench.clock_scaled(0.6, None) is None
 
 
 def test_nvml_sampler_keeps_only_the_marked_window():
