@@ -403,14 +403,15 @@ int fwd_common(const void* Q, const void* K, const void* V, void* O, float* LSE,
   if (dtype == FA_FP32) {
     e = launch_fwd_f32(static_cast<const float*>(Q), static_cast<const float*>(K), static_cast<const float*>(V), a, s);
   } else {
-    CUtensorMap tq, tk, tv;
+    CUtensorMap tq, tk, tv, to;
     CUresult r;
     if ((r = make_tile_map(&tq, Q, B, N, H, d, 128)) != CUDA_SUCCESS ||
         (r = make_tile_map(&tk, K, B, N, Hkv, d, 128)) != CUDA_SUCCESS ||
-        (r = make_tile_map(&tv, V, B, N, Hkv, d, 128)) != CUDA_SUCCESS)
+        (r = make_tile_map(&tv, V, B, N, Hkv, d, 128)) != CUDA_SUCCESS ||
+        (r = make_tile_map(&to, O, B, N, H, d, 128)) != CUDA_SUCCESS)
       return fail_encode(r);
     if (t_ev_start) cudaEventRecord(t_ev_start, s);
-    e = launch_fwd_bf16(tq, tk, tv, a, make_ctl(*st), s);
+    e = launch_fwd_bf16(tq, tk, tv, to, a, make_ctl(*st), s);
     if (t_ev_stop && e == cudaSuccess) cudaEventRecord(t_ev_stop, s);
   }
   if (e != cudaSuccess) return fail_cuda(e);

@@ -168,19 +168,6 @@ static_assert(BwdCfg::kOffDQS % 1024 == 0 && BwdCfg::kSmemBytes <= 232448, "shar
 
 __device__ __forceinline__ bool warp_all(bool ok) { return __all_sync(0xffffffffu, ok); }
 
-// TMA reduce-add of a shared-memory tile into global memory (fp32), and the
-// bulk-group bookkeeping around it.
-__device__ __forceinline__ void tma_reduce_add_4d(const CUtensorMap* map, const void* src, int c0, int c1, int c2,
-                                                  int c3) {
-  asm volatile(
-      "cp.reduce.async.bulk.tensor.4d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::"l"(
-          reinterpret_cast<uint64_t>(map)),
-      "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
-      : "memory");
-}
-__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
-__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 // TMEM column of the bf16 pairs for reduction step kk (16 query columns) of a
 // P^T / dS^T tile written by the two compute warpgroups.
@@ -204,10 +191,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = warp_id();
   const int lane = lane_id();
 
-  const int jt = blockIdx.x;                // key tile
-  const int hk = blockIdx.y / a.splits;     // K/V head
-  const int sp = blockIdx.y % a.splits;     // part of this key tile's walk
-  const int b = blockIdx.z;
+  // Key tile, K/V head, part of the key tile's walk, batch.  Causal: the
+  // launch order (block x fastest, then y, then z) is longest first over every
+  // (b, K/V head, part): the CTA's rank in it picks the key tile from the start
+  // of the sequence (whose walks are longest), the rest vary fastest.
+  int jt = static_cast<int>(blockIdx.x), y = static_cast<int>(blockIdx.y), b = static_cast<int>(blockIdx.z);
+  if (a.causal) {
+    const int yz = static_cast<int>(gridDim.y * gridDim.z);
+    const int rank = static_cast<int>(blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z));
+    jt = rank / yz;
+    y = (rank % yz) % static_cast<int>(gridDim.y);
+    b = (rank % yz) / static_cast<int>(gridDim.y);
+  }
+  const int hk = y / a.splits;  // K/V head
+  const int sp = y % a.splits;  // part of this key tile's walk
   const int key0 = jt * kBN;
   const int nq_total = (a.N + kBMq - 1) / kBMq;
   // query tiles holding every query that sees one of these keys:

@@ -26,13 +26,16 @@
 //     tile can see are never loaded or multiplied ("Flash Attention"
 //     (karlkratz.de), "Sliding Window Attention": blocks outside the window
 //     are skipped); only the tiles that straddle the window's edge are masked;
-//     under the causal mask CTAs with longer rows start first;
+//     under the causal mask the launch order is longest first over every
+//     (b, h): the CTAs of the last query tiles of all heads go first;
 //   * block-sparse masks (the kSparse instantiation): the CTA compacts the key
 //     tiles either query tile keeps into a list in shared memory; the loader
 //     streams only those, and each tile skips the ones it does not keep; a
 //     row that keeps none gets O = 0, LSE = -inf;
 //   * grouped-query attention: query head h reads K/V head h / (H / Hkv);
-//   * epilogue: O / l -> bf16 with 16-byte stores, LSE = (m + log2 l) ln 2.
+//   * epilogue: O / l -> bf16, staged in the query tile's shared memory (free
+//     once its last S MMA is done) in the 128-byte swizzled layout and written
+//     by TMA tile stores (whole coalesced lines); LSE = (m + log2 l) ln 2.
 // The two query tiles ping-pong: while the softmax of one tile runs, the
 // tensor pipe computes the other tile's products.
 #include <cuda_bf16.h>
@@ -89,6 +92,7 @@ struct FwdBars {
   uint64_t k_full[4], k_empty[4], v_full[4], v_empty[4];
   uint64_t s_full[2], p_full[2], o_done[2];
   uint64_t drain;
+  uint64_t epi[2];  // query tile t's O rows are staged in shared memory
   uint32_t tmem_base;
   int abort;
 };
@@ -98,7 +102,8 @@ __device__ __forceinline__ bool warp_all(bool ok) { return __all_sync(0xffffffff
 template <int D, bool kSparse>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                    const __grid_constant__ CUtensorMap tmV, const FwdArgs a, const DevCtl ctl) {
+                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO, const FwdArgs a,
+                    const DevCtl ctl) {
   using C = FwdCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -107,10 +112,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int lane = lane_id();
 
   // ---- work of this CTA ----
+  // Causal: the launch order (block x fastest, then y, then z) is longest
+  // first over every (b, h): the CTA's rank in that order picks the pair of
+  // query tiles from the end of the sequence, the head and batch vary fastest.
   const int nqb = gridDim.x;
-  const int cb = a.causal ? (nqb - 1 - static_cast<int>(blockIdx.x)) : static_cast<int>(blockIdx.x);
-  const int h = blockIdx.y;
-  const int b = blockIdx.z;
+  int cb = static_cast<int>(blockIdx.x), h = static_cast<int>(blockIdx.y), b = static_cast<int>(blockIdx.z);
+  if (a.causal) {
+    const int hb = static_cast<int>(gridDim.y * gridDim.z);
+    const int rank = static_cast<int>(blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z));
+    cb = nqb - 1 - rank / hb;
+    h = (rank % hb) % static_cast<int>(gridDim.y);
+    b = (rank % hb) / static_cast<int>(gridDim.y);
+  }
   const int hk = h / (a.H / a.Hkv);  // K/V head of this query head (grouped-query attention)
   // Key tiles [klo[t], klo[t] + nkt[t]) hold every key some row of query tile
   // t may see; the CTA streams their union, key tiles kbase .. kbase + nk - 1
@@ -193,6 +206,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars->s_full[t], 1);
       mbar_init(&bars->p_full[t], kBM);
       mbar_init(&bars->o_done[t], 1);
+      mbar_init(&bars->epi[t], kBM);
     }
     mbar_init(&bars->drain, 1);
     bars->abort = (*reinterpret_cast<volatile unsigned int*>(ctl.abort_epoch) == ctl.epoch) ? 1 : 0;
@@ -322,10 +336,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ok && nkt[t] > 0) {
         ok = warp_all(wait_bar(&bars->o_done[t], (nkt[t] - 1) & 1, w, 9));
         if (ok) {
+          // O_t / l as bf16 into Q_t's shared memory: every S_t MMA, issued
+          // before the last P_t V, has completed when o_done fires.  Row r
+          // writes its 16-byte units in the 128-byte swizzled [128][64]
+          // sub-tiles (eight rows of a quarter-warp hit eight distinct bank
+          // groups), then one thread stores the tile with TMA.
           tc_fence_after();
           const float inv = (l > 0.f) ? 1.f / l : 0.f;
-          __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.O) +
-                                ((static_cast<size_t>(b) * a.N + qrow) * a.H + h) * D;
+          uint8_t* stage = smem + C::kOffQ + t * C::kTileBytes;
 #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
             uint32_t o[32];
@@ -336,15 +354,23 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int i = 0; i < 16; ++i)
               pkd[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
-            if (qrow < a.N) {
+            const uint32_t sub = smem_u32(stage + (c >> 1) * C::kSubBytes);
 #pragma unroll
-              for (int i = 0; i < 4; ++i)
-                st_global_v4(orow + c * 32 + i * 8, pkd[4 * i], pkd[4 * i + 1], pkd[4 * i + 2], pkd[4 * i + 3]);
-            }
+            for (int i = 0; i < 4; ++i)
+              st_shared_v4(sub + sw128_offset(r, (c & 1) * 4 + i), pkd[4 * i], pkd[4 * i + 1], pkd[4 * i + 2],
+                           pkd[4 * i + 3]);
           }
+          fence_proxy_async_smem();
           if (qrow < a.N) {
             const float lse = (l > 0.f) ? (m + __log2f(l)) * 0.69314718055994531f : -INFINITY;
             a.LSE[(static_cast<size_t>(b) * a.H + h) * a.N + qrow] = lse;
+          }
+          mbar_arrive(&bars->epi[t]);
+          if (r == 0 && wait_bar(&bars->epi[t], 0, w, 10)) {
+            // rows past N are outside the tensor and are not written
+            for (int c = 0; c < C::kSub; ++c) tma_store_4d(&tmO, stage + c * C::kSubBytes, c * 64, q0[t], h, b);
+            bulk_commit();
+            bulk_wait_read_all();  // the staging tile is read before the CTA's shared memory is released
           }
         }
       }
@@ -473,14 +499,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace
 
-cudaError_t launch_fwd_bf16(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const FwdArgs& a,
-                            const DevCtl& c, cudaStream_t s) {
+cudaError_t launch_fwd_bf16(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& to,
+                            const FwdArgs& a, const DevCtl& c, cudaStream_t s) {
   const int nqb = (a.N + 2 * kBM - 1) / (2 * kBM);
   const dim3 grid(nqb, a.H, a.B);
   auto run = [&](auto kernel, int smem) -> cudaError_t {
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    kernel<<<grid, kThreads, smem, s>>>(tq, tk, tv, a, c);
+    kernel<<<grid, kThreads, smem, s>>>(tq, tk, tv, to, a, c);
     return cudaGetLastError();
   };
   const bool sparse = a.block_mask != nullptr;

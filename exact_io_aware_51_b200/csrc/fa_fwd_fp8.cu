@@ -46,6 +46,11 @@ static_assert(2 * kRegSoftmax + kRegOther == 3 * 168, "register split must match
 constexpr float kTau = 4.0f;   // lazy-rescale threshold (log2 units)
 constexpr float kPOff = 4.0f;  // P is stored as 2^(s - m + kPOff)
 static_assert(kTau + kPOff <= 8.0f, "p' = 2^(kTau + kPOff) must stay below the e4m3 maximum 448");
+// One score pair in kPolyEvery takes its exponentials on the FMA pipe
+// (exp2_poly2: range reduction and a degree-3 polynomial, relative error
+// 7.5e-5, far below e4m3's 2^-4) instead of the MUFU unit, which each score
+// otherwise needs once while the 8-bit MMAs take half the bf16 time.  0: none.
+constexpr int kPolyEvery = 0;
 
 struct Cfg {
   static constexpr int kTile = kBM * 128;  // one [128][128] e4m3 tile: 16 KB
@@ -87,9 +92,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int lane = lane_id();
 
   const int nqb = gridDim.x;
-  const int cb = a.causal ? (nqb - 1 - static_cast<int>(blockIdx.x)) : static_cast<int>(blockIdx.x);
-  const int h = blockIdx.y;
-  const int b = blockIdx.z;
+  // causal: longest first over every (b, h), as in the bf16 kernel
+  int cb = static_cast<int>(blockIdx.x), h = static_cast<int>(blockIdx.y), b = static_cast<int>(blockIdx.z);
+  if (a.causal) {
+    const int hb = static_cast<int>(gridDim.y * gridDim.z);
+    const int rank = static_cast<int>(blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z));
+    cb = nqb - 1 - rank / hb;
+    h = (rank % hb) % static_cast<int>(gridDim.y);
+    b = (rank % hb) / static_cast<int>(gridDim.y);
+  }
   const int hk = h / (a.H / a.Hkv);
   // key tiles [klo[t], klo[t] + nkt[t]) of query tile t; the CTA streams their union
   int q0[2], klo[2], nkt[2];
@@ -268,8 +279,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int c = q * 64 + 4 * i;
             const float2 x0 = ffma2(make_float2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sl2v, offv);
             const float2 x1 = ffma2(make_float2(__uint_as_float(sr[c + 2]), __uint_as_float(sr[c + 3])), sl2v, offv);
-            const float2 p0 = make_float2(ex2(x0.x), ex2(x0.y));
-            const float2 p1 = make_float2(ex2(x1.x), ex2(x1.y));
+            const bool poly0 = kPolyEvery > 0 && (2 * i) % (kPolyEvery > 0 ? kPolyEvery : 1) == kPolyEvery - 1;
+            const bool poly1 = kPolyEvery > 0 && (2 * i + 1) % (kPolyEvery > 0 ? kPolyEvery : 1) == kPolyEvery - 1;
+            const float2 p0 = poly0 ? exp2_poly2(x0) : make_float2(ex2(x0.x), ex2(x0.y));
+            const float2 p1 = poly1 ? exp2_poly2(x1) : make_float2(ex2(x1.x), ex2(x1.y));
             rs = fadd2(rs, fadd2(p0, p1));
             pk[i] = pack_e4m3x4(p0.x, p0.y, p1.x, p1.y);
           }

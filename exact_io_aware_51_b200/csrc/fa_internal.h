@@ -119,7 +119,7 @@ cudaError_t launch_decode(const CUtensorMap& tk, const CUtensorMap& tv, const De
 
 // Kernel launchers (each returns the cudaError_t of the launch).
 cudaError_t launch_fwd_bf16(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                            const FwdArgs& a, const DevCtl& c, cudaStream_t s);
+                            const CUtensorMap& to, const FwdArgs& a, const DevCtl& c, cudaStream_t s);
 cudaError_t launch_fwd_fp8(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const FwdArgs& a,
                            float out_scale, const DevCtl& c, cudaStream_t s);
 cudaError_t launch_fwd_f32(const float* Q, const float* K, const float* V, const FwdArgs& a, cudaStream_t s);
