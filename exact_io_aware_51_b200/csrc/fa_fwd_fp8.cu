@@ -50,7 +50,7 @@ static_assert(kTau + kPOff <= 8.0f, "p' = 2^(kTau + kPOff) must stay below the e
 // (exp2_poly2: range reduction and a degree-3 polynomial, relative error
 // 7.5e-5, far below e4m3's 2^-4) instead of the MUFU unit, which each score
 // otherwise needs once while the 8-bit MMAs take half the bf16 time.  0: none.
-constexpr int kPolyEvery = 0;
+constexpr int kPolyEvery = 8;
 
 struct Cfg {
   static constexpr int kTile = kBM * 128;  // one [128][128] e4m3 tile: 16 KB
