@@ -13,6 +13,7 @@ there is no CPU fallback.  If the library is missing, every call raises.
 from __future__ import annotations
 
 import ctypes
+import os
 import math
 import pathlib
 
@@ -57,7 +58,13 @@ class FAError(RuntimeError):
 
 
 def lib_path() -> pathlib.Path:
-    return _PKG / "libfa.so"
+    """The library the binding loads: ``libfa.so``, or the checking build
+    ``libfa_debug.so`` (device-side bounds checks, see ``fa_last_device_status``)
+    when the environment variable ``FA_LIBRARY`` names it."""
+    name = os.environ.get("FA_LIBRARY", "libfa.so")
+    if name not in ("libfa.so", "libfa_debug.so"):
+        raise FAError(-1, f"FA_LIBRARY={name!r}: expected libfa.so or libfa_debug.so")
+    return _PKG / name
 
 
 def lib() -> ctypes.CDLL:

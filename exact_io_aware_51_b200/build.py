@@ -1,9 +1,11 @@
 """Build the CUDA library ``libfa.so`` in-tree (sm_100a only).
 
 ``python -m exact_io_aware_51_b200.build`` compiles every ``csrc/*.cu`` with
-nvcc for ``sm_100a``: the product library ``exact_io_aware_51_b200/libfa.so``
-and, from ``fa_probe.cu`` alone, the test library ``libfa_probe.so`` (single
-MMA tile probes; declared in ``csrc/fa_testing.h``, not in the public header).
+nvcc for ``sm_100a``: the product library ``exact_io_aware_51_b200/libfa.so``;
+the checking build ``libfa_debug.so`` (the same sources with ``FA_DEBUG``:
+device-side bounds checks that record a status and skip the access); and, from
+``fa_probe.cu`` alone, the test library ``libfa_probe.so`` (single MMA tile
+probes; declared in ``csrc/fa_testing.h``, not in the public header).
 nvcc cross-compiles without a GPU.  The CUDA runtime is linked statically, so
 the libraries only need the driver at run time.
 """
@@ -28,6 +30,7 @@ SOURCES = ("fa_api.cu", "fa_fwd_bf16.cu", "fa_fwd_fp8.cu", "fa_fwd_f32.cu", "fa_
            "fa_bwd64.cu", "fa_decode.cu")
 PROBE_SOURCES = ("fa_probe.cu",)
 PROBE_LIB = PKG / "libfa_probe.so"
+DEBUG_LIB = PKG / "libfa_debug.so"
 ARCH = ("-gencode", "arch=compute_100a,code=sm_100a")
 FLAGS = ("-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall",
          "--expt-relaxed-constexpr")
@@ -46,15 +49,17 @@ def _deps():
 
 
 def up_to_date() -> bool:
-    if not LIB.exists() or not PROBE_LIB.exists():
+    libs = (LIB, PROBE_LIB, DEBUG_LIB)
+    if not all(p.exists() for p in libs):
         return False
-    t = min(LIB.stat().st_mtime, PROBE_LIB.stat().st_mtime)
+    t = min(p.stat().st_mtime for p in libs)
     return all(p.stat().st_mtime <= t for p in _deps())
 
 
-def _compile(src: pathlib.Path, verbose: bool) -> pathlib.Path:
-    obj = BUILD / (src.stem + ".o")
-    cmd = [nvcc(), *ARCH, *FLAGS, "-I", str(INCLUDE), "-I", str(CSRC), "-c", str(src), "-o", str(obj)]
+def _compile(src: pathlib.Path, verbose: bool, debug: bool = False) -> pathlib.Path:
+    obj = BUILD / (src.stem + ("_debug.o" if debug else ".o"))
+    cmd = [nvcc(), *ARCH, *FLAGS, *(("-DFA_DEBUG",) if debug else ()), "-I", str(INCLUDE), "-I", str(CSRC), "-c",
+           str(src), "-o", str(obj)]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
         print(" ".join(cmd), flush=True)
@@ -71,12 +76,12 @@ def build(force: bool = False, verbose: bool = False) -> pathlib.Path:
     if not force and up_to_date():
         return LIB
     BUILD.mkdir(exist_ok=True)
-    every = SOURCES + PROBE_SOURCES
-    with concurrent.futures.ThreadPoolExecutor(max_workers=len(every)) as ex:
-        objs = dict(zip(every, ex.map(lambda s: _compile(CSRC / s, verbose), every)))
-    for lib, srcs in ((LIB, SOURCES), (PROBE_LIB, PROBE_SOURCES)):
+    jobs = [(s, False) for s in SOURCES + PROBE_SOURCES] + [(s, True) for s in SOURCES]
+    with concurrent.futures.ThreadPoolExecutor(max_workers=len(jobs)) as ex:
+        objs = dict(zip(jobs, ex.map(lambda j: _compile(CSRC / j[0], verbose, j[1]), jobs)))
+    for lib, srcs, debug in ((LIB, SOURCES, False), (PROBE_LIB, PROBE_SOURCES, False), (DEBUG_LIB, SOURCES, True)):
         tmp = lib.with_suffix(".so.tmp")
-        cmd = [nvcc(), *ARCH, "-shared", "-o", str(tmp), *(str(objs[s]) for s in srcs), "-cudart", "static"]
+        cmd = [nvcc(), *ARCH, "-shared", "-o", str(tmp), *(str(objs[(s, debug)]) for s in srcs), "-cudart", "static"]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"link of {lib.name} failed:\n{r.stdout}\n{r.stderr}")

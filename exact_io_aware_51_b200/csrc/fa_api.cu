@@ -322,6 +322,7 @@ const char* fa_status_string(int status) {
     case FA_ERR_DEVICE_TIMEOUT: return "a kernel wait exceeded its limit; outputs of that launch are undefined";
     case FA_ERR_TOO_LARGE: return "problem exceeds a size limit";
     case FA_ERR_DEVICE_INPUT: return "device-side input out of range (sequence length or page index)";
+    case FA_ERR_DEVICE_CHECK: return "a device-side bounds check of the checking build failed";
     default: return "unknown status";
   }
 }
@@ -352,6 +353,7 @@ int fa_last_device_status(void* stream, int* detail) {
   e = cudaMemcpy(st->status, &zero, sizeof(int), cudaMemcpyHostToDevice);
   if (e != cudaSuccess) return fail_cuda(e);
   if (detail) *detail = v;
+  if (v & kDevCheck) return FA_ERR_DEVICE_CHECK;
   if (v & kDevBadInput) return FA_ERR_DEVICE_INPUT;
   return v ? FA_ERR_DEVICE_TIMEOUT : FA_OK;
 }

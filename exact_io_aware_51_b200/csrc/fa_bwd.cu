@@ -512,7 +512,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           fence_proxy_async_smem();
           if (!(ok = drain_sync())) break;
           if (issuer) {
-            tma_reduce_add_4d(&tmDQ, stage, 0, q0 + 64 * half, hq, b);
+            if (fa_dbg(q0 >= 0 && q0 < a.N && hq < a.H, ctl.status, 0x14))
+              tma_reduce_add_4d(&tmDQ, stage, 0, q0 + 64 * half, hq, b);
             bulk_commit();
           }
         }
@@ -535,7 +536,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_prefetch_desc(&tmV);
         tma_prefetch_desc(&tmDO);
         mbar_arrive_expect_tx(&bars->kv_full, 2 * C::kTile);
-        for (int c = 0; c < D / 64; ++c) {
+        const bool kv_ok = fa_dbg(key0 >= 0 && key0 < a.N && hk < a.Hkv && b < a.B, ctl.status, 0x11);
+        for (int c = 0; kv_ok && c < D / 64; ++c) {
           tma_load_4d(smem + C::kOffK + c * C::kSub, &tmK, &bars->kv_full, c * 64, key0, hk, b);
           tma_load_4d(smem + C::kOffV + c * C::kSub, &tmV, &bars->kv_full, c * 64, key0, hk, b);
         }
@@ -573,14 +575,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           if constexpr (kSparse) bars->info_q0[i & 3] = q0;
           const size_t bh = static_cast<size_t>(b) * a.H + hq_i;
           mbar_arrive_expect_tx(&bars->q_full[st], 2 * C::kTile + 1024);
-          for (int c = 0; c < D / 64; ++c) {
+          // the tile's rows and head exist, and its 128 LSE / D entries lie inside the [B, H, Npad] rows
+          const bool q_ok = fa_dbg(q0 >= 0 && q0 < a.N && hq_i >= hk * G && hq_i < hk * G + G && hq_i < a.H,
+                                   ctl.status, 0x12) &&
+                            fa_dbg(bh * a.Npad + q0 + kBMq <= static_cast<size_t>(a.B) * a.H * a.Npad, ctl.status,
+                                   0x13);
+          for (int c = 0; q_ok && c < D / 64; ++c) {
             tma_load_4d(smem + C::kOffQ + st * C::kTile + c * C::kSub, &tmQ, &bars->q_full[st], c * 64, q0, hq_i,
                         b);
             tma_load_4d(smem + C::kOffDO + st * C::kTile + c * C::kSub, &tmDO, &bars->q_full[st], c * 64, q0, hq_i,
                         b);
           }
-          bulk_load(smem + C::kOffL + st * 512, a.LSE2 + bh * a.Npad + q0, 512, &bars->q_full[st]);
-          bulk_load(smem + C::kOffDv + st * 512, a.Dvec + bh * a.Npad + q0, 512, &bars->q_full[st]);
+          if (q_ok) {
+            bulk_load(smem + C::kOffL + st * 512, a.LSE2 + bh * a.Npad + q0, 512, &bars->q_full[st]);
+            bulk_load(smem + C::kOffDv + st * 512, a.Dvec + bh * a.Npad + q0, 512, &bars->q_full[st]);
+          }
           ++q_issued;
         }
         // teardown: no copy of this CTA may still be writing its shared memory
@@ -596,18 +605,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t sDO = smem_u32(smem + C::kOffDO);
         // S^T = K Q^T (or dP^T = V dO^T): A [128 keys][128 d] K-major, B [128 q][128 d] K-major
         auto issue_s = [&](uint32_t a_base, uint32_t b_base, uint32_t col) {
+          const uint64_t ad = sw128_desc(a_base, 16, 1024), bd = sw128_desc(b_base, 16, 1024);
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * C::kSub + (kk & 3) * 32;
-            umma_ss(tmem + col, sw128_desc(a_base + off, 16, 1024), sw128_desc(b_base + off, 16, 1024), C::kIdescS,
-                    kk > 0 ? 1u : 0u);
+            const uint32_t off = ((kk >> 2) * C::kSub + (kk & 3) * 32) >> 4;
+            umma_ss(tmem + col, ad + off, bd + off, C::kIdescS, kk > 0 ? 1u : 0u);
           }
         };
         // dV += P^T dO (or dK += dS^T Q): A from TMEM (bf16 pairs), B [128 q][128 d] MN-major
         auto issue_kv = [&](uint32_t a_col, uint32_t b_base, uint32_t d_col, bool acc) {
+          const uint64_t bd = sw128_desc(b_base, C::kSub, 1024);
 #pragma unroll
           for (int kk = 0; kk < kBMq / 16; ++kk)
-            umma_ts(tmem + d_col, tmem + a_col + ts_col(kk), sw128_desc(b_base + kk * 2048, C::kSub, 1024),
+            umma_ts(tmem + d_col, tmem + a_col + ts_col(kk), bd + static_cast<uint32_t>(kk * 2048 >> 4),
                     C::kIdescKV, (acc || kk > 0) ? 1u : 0u);
         };
         bool ok = wait_bar(&bars->kv_full, 0, w, 11) && wait_bar(&bars->q_full[0], 0, w, 12);
@@ -642,10 +652,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           // dQ^T = K^T dS^T over R2: A = K as [128 d (M, contiguous)][128 keys], B = dS^T as
           // [128 q (N, contiguous)][128 keys] in the dO stage buffer
           const uint32_t ds = sDO + st * C::kTile;
+          const uint64_t kd = sw128_desc(sK, C::kSub, 1024), dsd = sw128_desc(ds, C::kSub, 1024);
 #pragma unroll
           for (int kk = 0; kk < kBN / 16; ++kk)
-            umma_ss(tmem + C::kColR2, sw128_desc(sK + kk * 2048, C::kSub, 1024),
-                    sw128_desc(ds + kk * 2048, C::kSub, 1024), C::kIdescQ, kk > 0 ? 1u : 0u);
+            umma_ss(tmem + C::kColR2, kd + static_cast<uint32_t>(kk * 2048 >> 4),
+                    dsd + static_cast<uint32_t>(kk * 2048 >> 4), C::kIdescQ, kk > 0 ? 1u : 0u);
           umma_commit(&bars->dq_full);
           umma_commit(&bars->q_empty[st]);
           if (more) {

@@ -414,8 +414,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_prefetch_desc(&tmV);
         tma_prefetch_desc(&tmDO);
         mbar_arrive_expect_tx(&bars->kv_full, 2 * C::kTile);
-        tma_load_4d(smem + C::kOffK, &tmK, &bars->kv_full, 0, key0, hk, b);
-        tma_load_4d(smem + C::kOffV, &tmV, &bars->kv_full, 0, key0, hk, b);
+        if (fa_dbg(key0 >= 0 && key0 < a.N && hk < a.Hkv && b < a.B, ctl.status, 0x31)) {
+          tma_load_4d(smem + C::kOffK, &tmK, &bars->kv_full, 0, key0, hk, b);
+          tma_load_4d(smem + C::kOffV, &tmV, &bars->kv_full, 0, key0, hk, b);
+        }
         int qt = qt_beg, hq = hq_beg;
         if constexpr (kSparse) {
           qt = i0;
@@ -449,10 +451,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           if constexpr (kSparse) bars->info_q0[i & 3] = q0;
           const size_t bh = static_cast<size_t>(b) * a.H + hq_i;
           mbar_arrive_expect_tx(&bars->q_full[st], 2 * C::kTile + 1024);
-          tma_load_4d(smem + C::kOffQ + st * C::kTile, &tmQ, &bars->q_full[st], 0, q0, hq_i, b);
-          tma_load_4d(smem + C::kOffDO + st * C::kTile, &tmDO, &bars->q_full[st], 0, q0, hq_i, b);
-          bulk_load(smem + C::kOffL + st * 512, a.LSE2 + bh * a.Npad + q0, 512, &bars->q_full[st]);
-          bulk_load(smem + C::kOffDv + st * 512, a.Dvec + bh * a.Npad + q0, 512, &bars->q_full[st]);
+          if (fa_dbg(q0 >= 0 && q0 < a.N && hq_i < a.H &&
+                         bh * a.Npad + q0 + kBMq <= static_cast<size_t>(a.B) * a.H * a.Npad,
+                     ctl.status, 0x32)) {
+            tma_load_4d(smem + C::kOffQ + st * C::kTile, &tmQ, &bars->q_full[st], 0, q0, hq_i, b);
+            tma_load_4d(smem + C::kOffDO + st * C::kTile, &tmDO, &bars->q_full[st], 0, q0, hq_i, b);
+            bulk_load(smem + C::kOffL + st * 512, a.LSE2 + bh * a.Npad + q0, 512, &bars->q_full[st]);
+            bulk_load(smem + C::kOffDv + st * 512, a.Dvec + bh * a.Npad + q0, 512, &bars->q_full[st]);
+          }
           ++q_issued;
         }
         // teardown: no copy of this CTA may still be writing its shared memory

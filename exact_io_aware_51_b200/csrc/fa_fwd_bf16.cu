@@ -361,14 +361,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                            pkd[4 * i + 3]);
           }
           fence_proxy_async_smem();
-          if (qrow < a.N) {
+          if (qrow < a.N && fa_dbg(b < a.B && h < a.H, ctl.status, 0x04)) {
             const float lse = (l > 0.f) ? (m + __log2f(l)) * 0.69314718055994531f : -INFINITY;
             a.LSE[(static_cast<size_t>(b) * a.H + h) * a.N + qrow] = lse;
           }
           mbar_arrive(&bars->epi[t]);
           if (r == 0 && wait_bar(&bars->epi[t], 0, w, 10)) {
             // rows past N are outside the tensor and are not written
-            for (int c = 0; c < C::kSub; ++c) tma_store_4d(&tmO, stage + c * C::kSubBytes, c * 64, q0[t], h, b);
+            if (fa_dbg(q0[t] >= 0 && q0[t] < a.N, ctl.status, 0x03))
+              for (int c = 0; c < C::kSub; ++c) tma_store_4d(&tmO, stage + c * C::kSubBytes, c * 64, q0[t], h, b);
             bulk_commit();
             bulk_wait_read_all();  // the staging tile is read before the CTA's shared memory is released
           }
@@ -388,6 +389,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive_expect_tx(&bars->q_full, qbytes);
         for (int t = 0; t < 2; ++t) {
           if (nkt[t] == 0) continue;
+          if (!fa_dbg(q0[t] >= 0 && q0[t] < a.N && h < a.H && b < a.B, ctl.status, 0x01)) continue;
           for (int c = 0; c < C::kSub; ++c)
             tma_load_4d(smem + C::kOffQ + t * C::kTileBytes + c * C::kSubBytes, &tmQ, &bars->q_full, c * 64,
                         q0[t], h, b);
@@ -398,16 +400,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int n = j / C::kStages;
           if (j >= C::kStages && !wait_bar(&bars->k_empty[s], (n - 1) & 1, w, 1)) break;
           const uint32_t extra = (ctl.inject == 1 && j == 0) ? 16u : 0u;  // test-only: never completes
+          int krow = stream_tile(j) * kBN;
+#ifdef FA_DEBUG
+          if (ctl.inject == 2 && j == 0) krow += a.N;  // test-only: a key row the check must refuse
+#endif
+          const bool kv_ok = fa_dbg(krow >= 0 && krow < a.N && hk < a.Hkv && b < a.B, ctl.status, 0x02);
           mbar_arrive_expect_tx(&bars->k_full[s], C::kTileBytes + extra);
-          for (int c = 0; c < C::kSub; ++c)
+          for (int c = 0; kv_ok && c < C::kSub; ++c)
             tma_load_4d(smem + C::kOffK + s * C::kTileBytes + c * C::kSubBytes, &tmK, &bars->k_full[s], c * 64,
-                        stream_tile(j) * kBN, hk, b);
+                        krow, hk, b);
           ++k_issued;
           if (j >= C::kStages && !wait_bar(&bars->v_empty[s], (n - 1) & 1, w, 2)) break;
           mbar_arrive_expect_tx(&bars->v_full[s], C::kTileBytes);
-          for (int c = 0; c < C::kSub; ++c)
+          for (int c = 0; kv_ok && c < C::kSub; ++c)
             tma_load_4d(smem + C::kOffV + s * C::kTileBytes + c * C::kSubBytes, &tmV, &bars->v_full[s], c * 64,
-                        stream_tile(j) * kBN, hk, b);
+                        krow, hk, b);
           ++v_issued;
         }
         // teardown: no copy of this CTA may still be writing its shared memory

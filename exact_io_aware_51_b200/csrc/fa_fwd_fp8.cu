@@ -343,18 +343,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int t = 0; t < 2; ++t) qbytes += (nkt[t] > 0) ? C::kTile : 0;
         mbar_arrive_expect_tx(&bars->q_full, qbytes);
         for (int t = 0; t < 2; ++t)
-          if (nkt[t] > 0) tma_load_4d(smem + C::kOffQ + t * C::kTile, &tmQ, &bars->q_full, 0, q0[t], h, b);
+          if (nkt[t] > 0 && fa_dbg(q0[t] >= 0 && q0[t] < a.N && h < a.H && b < a.B, ctl.status, 0x21))
+            tma_load_4d(smem + C::kOffQ + t * C::kTile, &tmQ, &bars->q_full, 0, q0[t], h, b);
         int k_issued = 0, v_issued = 0;
         for (int j = 0; j < nk; ++j) {
           const int s = j % C::kStages;
           const int n = j / C::kStages;
           if (j >= C::kStages && !wait_bar(&bars->k_empty[s], (n - 1) & 1, w, 1)) break;
           mbar_arrive_expect_tx(&bars->k_full[s], C::kTile);
-          tma_load_4d(smem + C::kOffK + s * C::kTile, &tmK, &bars->k_full[s], 0, stream_tile(j) * kBN, hk, b);
+          const int krow = stream_tile(j) * kBN;
+          const bool kv_ok = fa_dbg(krow >= 0 && krow < a.N && hk < a.Hkv && b < a.B, ctl.status, 0x22);
+          if (kv_ok) tma_load_4d(smem + C::kOffK + s * C::kTile, &tmK, &bars->k_full[s], 0, krow, hk, b);
           ++k_issued;
           if (j >= C::kStages && !wait_bar(&bars->v_empty[s], (n - 1) & 1, w, 2)) break;
           mbar_arrive_expect_tx(&bars->v_full[s], C::kTile);
-          tma_load_4d(smem + C::kOffV + s * C::kTile, &tmV, &bars->v_full[s], 0, stream_tile(j) * kBN, hk, b);
+          if (kv_ok) tma_load_4d(smem + C::kOffV + s * C::kTile, &tmV, &bars->v_full[s], 0, krow, hk, b);
           ++v_issued;
         }
         // teardown: no copy of this CTA may still be writing its shared memory

@@ -90,6 +90,21 @@ CUresult make_dq_accum_map_sw128(CUtensorMap* map, float* base, int B, int N, in
 // Status-word bit a kernel sets when device-side input data (a sequence length
 // or a page index) is out of range; the low bits name the check.
 constexpr int kDevBadInput = 0x2000;
+constexpr int kDevCheck = 0x4000;    // | check id: a bounds check of the FA_DEBUG build failed
+
+// Bounds and alignment checks of the checking build (compiled with FA_DEBUG):
+// fa_dbg(cond, status, id) is true when the access may go ahead; when cond is
+// false it records kDevCheck | id in the status word (first problem wins) and
+// the caller skips the access, so nothing traps or faults.  Without FA_DEBUG
+// it is the constant true and costs nothing.
+#ifdef FA_DEBUG
+__device__ __forceinline__ bool fa_dbg(bool cond, int* status, int id) {
+  if (!cond) atomicCAS(status, 0, kDevCheck | id);
+  return cond;
+}
+#else
+__device__ __forceinline__ constexpr bool fa_dbg(bool, int*, int) { return true; }
+#endif
 
 // One decode step over a paged KV cache: Q [B, H, d] (one query per sequence),
 // K, V pools [num_pages, page_size, Hkv, d], block_table [B, max_pages],

@@ -6,7 +6,10 @@
  * In libfa.so (the product library):
  *   fa_debug_inject: 1 makes the next forward launches' first key-tile
  *     barrier expect 16 bytes that never arrive, so its waits expire and the
- *     launch reports FA_ERR_DEVICE_TIMEOUT; 0 turns it off (process-wide).
+ *     launch reports FA_ERR_DEVICE_TIMEOUT; 2 (honoured only by the checking
+ *     build libfa_debug.so) moves the forward's first key-tile row past N, so
+ *     the loader's bounds check refuses the load and the launch reports
+ *     FA_ERR_DEVICE_CHECK; 0 turns it off (process-wide).
  *
  * In libfa_probe.so (a separate test library built from fa_probe.cu):
  *   fa_debug_umma: one 128 x N x K tcgen05 MMA tile, D = A B^T, with A [128][K]

@@ -64,7 +64,8 @@ enum {
   FA_ERR_LAUNCH = -6,          /* a CUDA call failed; see fa_last_cuda_error() */
   FA_ERR_DEVICE_TIMEOUT = -7,  /* a kernel's bounded wait expired (see fa_last_device_status) */
   FA_ERR_TOO_LARGE = -8,       /* a size limit above is exceeded */
-  FA_ERR_DEVICE_INPUT = -9     /* a kernel found device-side input out of range (see fa_last_device_status) */
+  FA_ERR_DEVICE_INPUT = -9,    /* a kernel found device-side input out of range (see fa_last_device_status) */
+  FA_ERR_DEVICE_CHECK = -10    /* a debug build's device-side bounds check failed (see fa_last_device_status) */
 };
 
 /*
@@ -346,10 +347,14 @@ int fa_last_cuda_error(void);
  * word.  Returns FA_OK if no kernel reported a problem since the last call,
  * FA_ERR_DEVICE_INPUT if a kernel found device-side input out of range
  * (fa_decode_paged), FA_ERR_DEVICE_TIMEOUT if a bounded wait expired (the
- * affected launch's outputs are then undefined), or FA_ERR_LAUNCH.  *detail
+ * affected launch's outputs are then undefined), FA_ERR_DEVICE_CHECK if a
+ * kernel of the checking build (libfa_debug.so, compiled with FA_DEBUG) found
+ * an index, coordinate or tensor-memory column outside its buffer (it skipped
+ * that access; the launch's outputs are undefined), or FA_ERR_LAUNCH.  *detail
  * (if not NULL) receives the raw word: 0x1000 | the id of the wait that
- * expired, or 0x2000 | the id of the failed input check (0xD1 a sequence
- * length, 0xD2 a page index).
+ * expired, 0x2000 | the id of the failed input check (0xD1 a sequence
+ * length, 0xD2 a page index), or 0x4000 | the id of the failed bounds check.
+ * The first problem recorded wins.
  */
 int fa_last_device_status(void* stream, int* detail);
 

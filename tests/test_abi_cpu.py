@@ -64,8 +64,18 @@ def test_test_only_symbols_live_outside_the_public_header(L):
     assert probe.fa_debug_umma(None, None, None, 64, 64, 0, 0, 0, None) == -1
 
 
+def test_checking_build_exports_the_same_symbols(L):
+    """libfa_debug.so (FA_DEBUG: device-side bounds checks) is the product
+    library compiled with the checks on: same exported entry points."""
+    def exported(path):
+        out = subprocess.run(["nm", "-D", "--defined-only", str(path)], capture_output=True, text=True,
+                             check=True).stdout
+        return set(re.findall(r" T (fa_[a-z0-9_]+)$", out, flags=re.M))
+    assert exported(fa.lib_path().parent / "libfa_debug.so") == exported(fa.lib_path())
+
+
 def test_status_strings(L):
-    for code in (0, -1, -2, -3, -4, -5, -6, -7, -8, -9):
+    for code in (0, -1, -2, -3, -4, -5, -6, -7, -8, -9, -10):
         assert fa.status_string(code) and "unknown" not in fa.status_string(code)
     assert "unknown" in fa.status_string(-99)
 
