@@ -22,7 +22,8 @@ import torch
 __all__ = [
     "FAError", "FA_BF16", "FA_FP32", "lib", "lib_path", "fwd", "fwd_fp8", "bwd", "bwd_workspace_size",
     "merge_partial", "accumulate", "cast_bf16", "decode_paged", "decode_workspace_size",
-    "last_device_status", "set_wait_limit_ms", "debug_inject", "debug_umma", "debug_umma_f8", "status_string",
+    "last_device_status", "set_wait_limit_ms", "debug_inject", "debug_umma", "debug_umma_f8", "debug_umma_2cta",
+    "status_string",
     "set_kernel_events",
     "attention", "EXPORTED",
 ]
@@ -42,7 +43,8 @@ EXPORTED = ("fa_fwd", "fa_bwd_workspace_size", "fa_bwd", "fa_status_string", "fa
             "fa_fwd_fp8_blocksparse")
 # Test-only symbols (csrc/fa_testing.h): the first in libfa.so, the others in the
 # separate test library libfa_probe.so.
-TESTING_EXPORTED = {"libfa.so": ("fa_debug_inject",), "libfa_probe.so": ("fa_debug_umma", "fa_debug_umma_f8")}
+TESTING_EXPORTED = {"libfa.so": ("fa_debug_inject",),
+                    "libfa_probe.so": ("fa_debug_umma", "fa_debug_umma_f8", "fa_debug_umma_2cta")}
 _PROBE = None
 
 
@@ -145,6 +147,8 @@ def probe_lib() -> ctypes.CDLL:
     P.fa_debug_umma.restype = i
     P.fa_debug_umma_f8.argtypes = [vp, vp, vp, i, i, i, vp]
     P.fa_debug_umma_f8.restype = i
+    P.fa_debug_umma_2cta.argtypes = [vp, vp, vp, i, i, i, i, vp, vp]
+    P.fa_debug_umma_2cta.restype = i
     _PROBE = P
     return P
 
@@ -447,6 +451,21 @@ def debug_umma_f8(a: torch.Tensor, b: torch.Tensor, b_mn_major: int, a_tmem: int
                                 _stream_handle(stream, a.device))
     if rc != 0:
         raise FAError(rc, "fa_debug_umma_f8")
+    return dmat
+
+
+def debug_umma_2cta(a: torch.Tensor, b: torch.Tensor, b_mn_major: int, a_tmem: int = 0, stream=None) -> torch.Tensor:
+    """One M = 256 tcgen05 tile over a two-CTA cluster, D = A B^T (test-only): a [256, K], b [128, K] bf16 cuda.
+    Raises if the MMAs did not complete."""
+    n, kdim = b.shape
+    dmat = torch.empty((256, n), dtype=torch.float32, device=a.device)
+    status = torch.zeros(1, dtype=torch.int32, device=a.device)
+    rc = probe_lib().fa_debug_umma_2cta(a.data_ptr(), b.data_ptr(), dmat.data_ptr(), n, kdim, int(b_mn_major),
+                                        int(a_tmem), status.data_ptr(), _stream_handle(stream, a.device))
+    if rc != 0:
+        raise FAError(rc, "fa_debug_umma_2cta")
+    if int(status.item()) != 0:
+        raise FAError(-7, "fa_debug_umma_2cta: the MMAs did not complete")
     return dmat
 
 

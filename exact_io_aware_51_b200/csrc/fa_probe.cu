@@ -213,6 +213,144 @@ __global__ void __launch_bounds__(128, 1)
   }
 }
 
+// ---------------------------------------------------------------------------
+// Two-CTA probe: one M = 256 tile over a cluster of two CTAs,
+// D[256][N] = A[256][K] * B[N][K]^T, with every tcgen05 instruction in its
+// cta_group::2 form.  CTA r holds rows [128 r, 128 r + 128) of A (in shared
+// memory, K-major, or in its tensor memory) and rows [r N/2, (r + 1) N/2) of B
+// (K-major, or MN-major with the N rows contiguous); CTA 0 issues the MMAs, the
+// commit arrives on the barrier of both CTAs, and each CTA reads its 128 rows
+// of D out of its own tensor memory.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(128, 1)
+    umma2_probe_kernel(const __nv_bfloat16* __restrict__ A, const __nv_bfloat16* __restrict__ B,
+                       float* __restrict__ D, int N, int K, int b_mn, int a_tmem, int* __restrict__ status) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;          // 128 x K bf16, up to 32 KB
+  uint8_t* sB = smem + 32768;  // N/2 x K bf16, up to 16 KB
+  __shared__ uint64_t bar;
+  __shared__ uint32_t tbase;
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int rank = static_cast<int>(cluster_rank());
+  const int nh = N / 2;
+  const __nv_bfloat16* Ar = A + static_cast<size_t>(rank) * 128 * K;
+  const __nv_bfloat16* Br = B + static_cast<size_t>(rank) * nh * K;
+
+  if (!a_tmem) {
+    for (int e = tid; e < 128 * K; e += 128) {
+      const int m = e / K, k = e % K;
+      *reinterpret_cast<__nv_bfloat16*>(sA + (k / 64) * (128 * 128) + sw128_offset(m, (k % 64) / 8) + (k % 8) * 2) =
+          Ar[e];
+    }
+  }
+  for (int e = tid; e < nh * K; e += 128) {
+    const int n = e / K, k = e % K;
+    uint32_t off;
+    if (b_mn == 0)
+      off = (k / 64) * (nh * 128) + sw128_offset(n, (k % 64) / 8) + (k % 8) * 2;
+    else  // nh = 64: one 64-element chunk per reduction row
+      off = sw128_offset(k, n / 8) + (n % 8) * 2;
+    *reinterpret_cast<__nv_bfloat16*>(sB + off) = Br[e];
+  }
+  if (tid == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(smem_u32(&tbase))
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tbase;
+  const uint32_t lane_bits = static_cast<uint32_t>(warp * 32) << 16;
+  if (a_tmem) {
+    // row 128 rank + tid into lane tid, two bf16 per column from column 256
+    for (int c0 = 0; c0 < K / 2; c0 += 16) {
+      uint32_t r[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int k = 2 * (c0 + i);
+        const __nv_bfloat162 v = __halves2bfloat162(Ar[tid * K + k], Ar[tid * K + k + 1]);
+        r[i] = *reinterpret_cast<const uint32_t*>(&v);
+      }
+      tmem_st16(tmem + lane_bits + 256 + c0, r);
+    }
+    tmem_wait_st();
+  }
+  // both CTAs' operands, barriers and tensor memory are in place
+  tc_fence_before();
+  cluster_sync_all();
+  tc_fence_after();
+
+  if (rank == 0 && tid == 0) {
+    const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sB);
+    const uint32_t idesc = idesc_bf16(256, N, 0, b_mn);
+    for (int kk = 0; kk < K / 16; ++kk) {
+      const uint64_t bd = (b_mn == 0) ? sw128_desc(b0 + (kk / 4) * (nh * 128) + (kk % 4) * 32, 16, 1024)
+                                      : sw128_desc(b0 + kk * 2048, 16, 1024);
+      const uint32_t acc = kk > 0 ? 1u : 0u;
+      if (a_tmem) {
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(tmem),
+            "r"(tmem + 256 + kk * 8), "l"(bd), "r"(idesc), "r"(acc)
+            : "memory");
+      } else {
+        const uint64_t ad = sw128_desc(a0 + (kk / 4) * (128 * 128) + (kk % 4) * 32, 16, 1024);
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem),
+            "l"(ad), "l"(bd), "r"(idesc), "r"(acc)
+            : "memory");
+      }
+    }
+    const uint16_t mask = 0x3;
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+            smem_u32(&bar)),
+        "h"(mask)
+        : "memory");
+  }
+  // bounded wait for the MMAs
+  const uint64_t t0 = globaltimer_ns();
+  bool done = false;
+  while (!(done = mbar_try_wait(&bar, 0)) && globaltimer_ns() - t0 < 2000000000ull) {
+  }
+  done = __all_sync(0xffffffffu, done);
+  if (!done && (tid & 31) == 0) atomicExch(status, 1);
+  tc_fence_after();
+  if (done) {
+    for (int c0 = 0; c0 < N; c0 += 32) {
+      uint32_t r[32];
+      tmem_ld32(tmem + lane_bits + c0, r);
+      tmem_wait_ld();
+      reg_fence32(r);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) D[(static_cast<size_t>(rank) * 128 + tid) * N + c0 + i] = __uint_as_float(r[i]);
+    }
+  }
+  // neither CTA frees its tensor memory while the pair's MMAs may still use it
+  tc_fence_before();
+  cluster_sync_all();
+  tc_fence_after();
+  if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, 512;" ::"r"(tmem) : "memory");
+}
+
 cudaError_t launch_umma_probe_f8(const void* A, const void* B, float* D, int N, int b_mn, int a_tmem,
                                  cudaStream_t s) {
   constexpr int smem = 32768 + 1024;
@@ -230,6 +368,16 @@ cudaError_t launch_umma_probe(const void* A, const void* B, float* D, int N, int
   if (e != cudaSuccess) return e;
   umma_probe_kernel<<<1, 128, smem, s>>>(static_cast<const __nv_bfloat16*>(A), static_cast<const __nv_bfloat16*>(B),
                                          D, N, K, a_mn, b_mn, a_tmem);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_umma2_probe(const void* A, const void* B, float* D, int N, int K, int b_mn, int a_tmem, int* status,
+                               cudaStream_t s) {
+  constexpr int smem = 49152 + 1024;
+  cudaError_t e = cudaFuncSetAttribute(umma2_probe_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  umma2_probe_kernel<<<2, 128, smem, s>>>(static_cast<const __nv_bfloat16*>(A), static_cast<const __nv_bfloat16*>(B),
+                                          D, N, K, b_mn, a_tmem, status);
   return cudaGetLastError();
 }
 
@@ -266,6 +414,17 @@ int fa_debug_umma_f8(const void* A, const void* B, float* D, int N, int b_mn_maj
   if (rc != FA_OK) return rc;
   const cudaError_t e =
       fa::launch_umma_probe_f8(A, B, D, N, b_mn_major ? 1 : 0, a_tmem ? 1 : 0, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
+}
+
+int fa_debug_umma_2cta(const void* A, const void* B, float* D, int N, int K, int b_mn_major, int a_tmem, int* status,
+                       void* stream) {
+  if (!A || !B || !D || !status) return FA_ERR_INVALID_ARG;
+  if (N != 128 || (K != 64 && K != 128)) return FA_ERR_UNSUPPORTED;
+  const int rc = fa::probe_device_ok();
+  if (rc != FA_OK) return rc;
+  const cudaError_t e = fa::launch_umma2_probe(A, B, D, N, K, b_mn_major ? 1 : 0, a_tmem ? 1 : 0, status,
+                                               static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
 }
 

@@ -23,6 +23,13 @@
  *     e4m3 bytes, D [128][N] fp32.  b_mn_major stores B with N contiguous;
  *     a_tmem reads A from tensor memory (four elements per column).  N must be
  *     64 or 128.
+ *   fa_debug_umma_2cta: one M = 256 tile over a cluster of two CTAs with every
+ *     tcgen05 instruction in its cta_group::2 form, D = A B^T with A [256][K],
+ *     B [N][K] bf16 and D [256][N] fp32.  CTA r holds A's rows [128 r, 128 r +
+ *     128) (K-major in shared memory, or in its tensor memory with a_tmem) and
+ *     B's rows [r N / 2, (r + 1) N / 2) (K-major, or N-contiguous with
+ *     b_mn_major).  N = 128, K = 64 or 128.  *status (device int) is set to 1
+ *     if the MMAs did not complete within 2 s.
  * Return values are the fa_status codes of include/fa.h.
  */
 #ifndef FA_TESTING_H
@@ -37,6 +44,8 @@ void fa_debug_inject(int mode);
 int fa_debug_umma(const void* A, const void* B, float* D, int N, int K, int a_mn_major, int b_mn_major,
                   int a_tmem, void* stream);
 int fa_debug_umma_f8(const void* A, const void* B, float* D, int N, int b_mn_major, int a_tmem, void* stream);
+int fa_debug_umma_2cta(const void* A, const void* B, float* D, int N, int K, int b_mn_major, int a_tmem, int* status,
+                       void* stream);
 
 #ifdef __cplusplus
 }

@@ -62,3 +62,23 @@ def test_umma_tile_e4m3(n, b_mn, a_tmem):
     # bound is 1e-3 (a wrong operand layout gives errors of order 1)
     ref = a.double().numpy() @ b.double().numpy().T
     assert rel_err(d.cpu(), ref) < 1e-3
+
+
+# Two-CTA tile (cta_group::2, M = 256 over a cluster of two CTAs, each holding
+# half of A's rows and half of B's rows): the forms a paired kernel would use for
+# S = Q K^T (both K-major), P V with P in each CTA's TMEM and V's feature halves
+# N-contiguous, and an MN-major B from shared memory.
+TWO_CTA_CASES = [(128, 0, 0), (64, 0, 0), (128, 1, 1), (128, 1, 0)]
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("k,b_mn,a_tmem", TWO_CTA_CASES)
+def test_umma_tile_two_cta(k, b_mn, a_tmem):
+    need_gpu()
+    g = torch.Generator().manual_seed(7000 + k * 10 + b_mn * 2 + a_tmem)
+    a = torch.randn(256, k, generator=g).to(torch.bfloat16)
+    b = torch.randn(128, k, generator=g).to(torch.bfloat16)
+    d = fa.debug_umma_2cta(a.cuda(), b.cuda(), b_mn, a_tmem)
+    torch.cuda.synchronize()
+    ref = a.double().numpy() @ b.double().numpy().T
+    assert rel_err(d.cpu(), ref) < 1e-5
