@@ -23,6 +23,7 @@ __all__ = [
     "FAError", "FA_BF16", "FA_FP32", "lib", "lib_path", "fwd", "fwd_fp8", "bwd", "bwd_workspace_size",
     "merge_partial", "accumulate", "cast_bf16", "decode_paged", "decode_workspace_size",
     "last_device_status", "set_wait_limit_ms", "debug_inject", "debug_umma", "debug_umma_f8", "debug_umma_2cta",
+    "debug_mma_rate",
     "status_string",
     "set_kernel_events",
     "attention", "EXPORTED",
@@ -44,7 +45,8 @@ EXPORTED = ("fa_fwd", "fa_bwd_workspace_size", "fa_bwd", "fa_status_string", "fa
 # Test-only symbols (csrc/fa_testing.h): the first in libfa.so, the others in the
 # separate test library libfa_probe.so.
 TESTING_EXPORTED = {"libfa.so": ("fa_debug_inject",),
-                    "libfa_probe.so": ("fa_debug_umma", "fa_debug_umma_f8", "fa_debug_umma_2cta")}
+                    "libfa_probe.so": ("fa_debug_umma", "fa_debug_umma_f8", "fa_debug_umma_2cta",
+                                       "fa_debug_mma_rate")}
 _PROBE = None
 
 
@@ -149,6 +151,8 @@ def probe_lib() -> ctypes.CDLL:
     P.fa_debug_umma_f8.restype = i
     P.fa_debug_umma_2cta.argtypes = [vp, vp, vp, i, i, i, i, vp, vp]
     P.fa_debug_umma_2cta.restype = i
+    P.fa_debug_mma_rate.argtypes = [i, i, i, i, i, vp, vp, vp, vp, vp]
+    P.fa_debug_mma_rate.restype = i
     _PROBE = P
     return P
 
@@ -467,6 +471,40 @@ def debug_umma_2cta(a: torch.Tensor, b: torch.Tensor, b_mn_major: int, a_tmem: i
     if int(status.item()) != 0:
         raise FAError(-7, "fa_debug_umma_2cta: the MMAs did not complete")
     return dmat
+
+
+MMA_RATE_KINDS = ("none", "tcgen05.ld", "tcgen05.st", "st.shared", "ld.shared", "bulk copy smem->global",
+                  "bulk reduce-add smem->global", "red.global.add.v4", "ld.global (L1)", "quad transpose + red.v4")
+
+
+def debug_mma_rate(mode: int, n: int, kind: int = 0, grid: int | None = None, reps: int = 1500, device=None) -> dict:
+    """Tensor-pipe rate probe (test-only): one CTA (mode 2: a CTA pair) per SM issues reps x 8 back-to-back
+    128 x n x 16 bf16 MMAs (mode 0: both operands in shared memory, 1: A in TMEM, 2: M = 256 over a CTA pair)
+    while four warps generate traffic of one kind (MMA_RATE_KINDS).  Returns the median SM clocks per MMA
+    instruction, per 128 x 128 x 16 of work on one SM, and the traffic warps' bytes per clock."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    if grid is None:
+        grid = torch.cuda.get_device_properties(dev).multi_processor_count
+        grid -= grid % 2
+    cyc = torch.zeros(grid, dtype=torch.int64, device=dev)
+    ops = torch.zeros(grid, dtype=torch.int64, device=dev)
+    scratch = torch.zeros(grid * 4 * 16384, dtype=torch.float32, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    rc = probe_lib().fa_debug_mma_rate(int(mode), int(n), int(kind), int(grid), int(reps), cyc.data_ptr(),
+                                       ops.data_ptr(), scratch.data_ptr(), status.data_ptr(), _stream_handle(None, dev))
+    if rc != 0:
+        raise FAError(rc, "fa_debug_mma_rate")
+    torch.cuda.synchronize(dev)
+    if int(status.item()) != 0:
+        raise FAError(-7, "fa_debug_mma_rate: the MMAs did not complete")
+    c = float(cyc.median().item())
+    o = float(ops.median().item())
+    per = c / (reps * 8)
+    m = 256 if mode == 2 else 128
+    ctas = 2 if mode == 2 else 1
+    return {"mode": mode, "n": n, "kind": MMA_RATE_KINDS[kind], "grid": grid, "clk_per_mma": per,
+            "clk_per_128x128x16": per * (128 * 128) / (m // ctas * n),
+            "traffic_bytes_per_clk": o * (16384.0 if kind == 9 else 4096.0) / c if kind else 0.0}
 
 
 class _Attention(torch.autograd.Function):

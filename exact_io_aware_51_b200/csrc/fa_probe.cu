@@ -381,6 +381,232 @@ cudaError_t launch_umma2_probe(const void* A, const void* B, float* D, int N, in
   return cudaGetLastError();
 }
 
+// ---------------------------------------------------------------------------
+// Tensor-pipe rate probe.  One CTA (or CTA pair, MODE 2) per SM: warp 0 issues
+// reps x 8 back-to-back 128 x N x 16 bf16 MMAs (256 x N x 16 for the pair)
+// into one TMEM accumulator and records the SM clocks until they complete.
+// Warps 4-7 can meanwhile load the SM with one kind of traffic and count
+// their 4 KB operations (the drain pattern, kind 9, counts 16 KB):
+//   1 tcgen05.ld, 2 tcgen05.st (TMEM columns 256-383), 3 st.shared,
+//   4 ld.shared, 5 bulk copy shared -> global, 6 bulk fp32 reduce-add
+//   shared -> global, 7 red.global.add.v4.f32 from registers, 8 ld.global
+//   (L1 hits), 9 a 4 x 4 transpose in lane quads then red.global.add.v4.f32.
+// Operand values are arbitrary: only the timing is read.
+// ---------------------------------------------------------------------------
+constexpr int kRateSmem = 200 * 1024;  // more than half the SM's shared memory: one CTA per SM
+
+template <int MODE>  // 0: A and B in shared memory, 1: A in TMEM, 2: CTA pair, both in shared memory
+__global__ void __launch_bounds__(256, 1)
+    mma_rate_kernel(int N, int reps, int kind, unsigned long long* __restrict__ cycles,
+                    unsigned long long* __restrict__ ops, float* __restrict__ scratch, int* __restrict__ status) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sA = smem_u32(smem);              // [128][128] bf16, two 16 KB K-chunks
+  const uint32_t sB = smem_u32(smem + 32768);      // up to [256][128] bf16, two K-chunks
+  const uint32_t sX = smem_u32(smem + 98304);      // 64 KB the traffic warps read and write
+  __shared__ uint64_t bar;
+  __shared__ uint32_t tbase;
+  __shared__ volatile int stop;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  for (int i = tid; i < 98304 / 4; i += 256)
+    reinterpret_cast<uint32_t*>(smem)[i] = 0x3c003c00u ^ ((static_cast<uint32_t>(i) * 2654435761u) & 0x00ff00ffu);
+  if (tid == 0) {
+    stop = 0;
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    if (MODE == 2) {
+      asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(smem_u32(&tbase))
+                   : "memory");
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+    } else {
+      tmem_alloc(&tbase, 512);
+    }
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tbase;
+  if (MODE == 1 && warp < 4) {  // A: 128 x 128 bf16 in TMEM columns 384..447
+    uint32_t r[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) r[i] = 0x3c003c00u ^ static_cast<uint32_t>(tid * 31 + i);
+    for (int c0 = 0; c0 < 64; c0 += 16) tmem_st16(tmem + (static_cast<uint32_t>(warp * 32) << 16) + 384 + c0, r);
+    tmem_wait_st();
+  }
+  tc_fence_before();
+  if (MODE == 2) cluster_sync_all(); else __syncthreads();
+  tc_fence_after();
+
+  const bool issuer = tid == 0 && (MODE != 2 || cluster_rank() == 0);
+  const unsigned long long c0 = clock64();
+  if (issuer) {
+    const int nb = (MODE == 2) ? N / 2 : N;  // B rows in this CTA
+    const uint32_t idesc = (MODE == 1) ? idesc_bf16(128, N, 0, 1) : idesc_bf16(MODE == 2 ? 256 : 128, N, 0, 0);
+    for (int r = 0; r < reps; ++r) {
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t acc = (r > 0 || kk > 0) ? 1u : 0u;
+        const uint64_t ad = sw128_desc(sA + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+        const uint64_t bd = sw128_desc(sB + (kk >> 2) * (nb * 128) + (kk & 3) * 32, 16, 1024);
+        if (MODE == 0) {
+          umma_ss(tmem, ad, bd, idesc, acc);
+        } else if (MODE == 1) {
+          // B MN-major: 16 K-rows of 128 bytes per step, N groups of 64 at 16 KB
+          umma_ts(tmem, tmem + 384 + kk * 8, sw128_desc(sB + kk * 2048, 16384, 1024), idesc, acc);
+        } else {
+          asm volatile(
+              "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+              "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem),
+              "l"(ad), "l"(bd), "r"(idesc), "r"(acc)
+              : "memory");
+        }
+      }
+    }
+    if (MODE == 2) {
+      const uint16_t mask = 0x3;
+      asm volatile(
+          "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+              smem_u32(&bar)),
+          "h"(mask)
+          : "memory");
+    } else {
+      umma_commit(&bar);
+    }
+  }
+  if (warp >= 4 && kind > 0) {
+    const int w4 = warp - 4;
+    const uint32_t lane_bits = static_cast<uint32_t>(w4 * 32) << 16;
+    float* mine = scratch + (static_cast<size_t>(blockIdx.x) * 4 + w4) * 16384;  // this warp's 64 KB
+    unsigned long long n = 0;
+    uint32_t acc = 0;
+    for (int it = 0; it < 200000 && !stop; ++it, ++n) {
+      if (kind == 1) {
+        uint32_t r[32];
+        tmem_ld32(tmem + lane_bits + 256 + (it & 3) * 32, r);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) acc += r[i];
+      } else if (kind == 2) {
+        uint32_t r[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) r[i] = static_cast<uint32_t>(it + i);
+        tmem_st32(tmem + lane_bits + 256 + (it & 3) * 32, r);
+        tmem_wait_st();
+      } else if (kind == 3 || kind == 4) {
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const uint32_t addr = sX + (((w4 * 8 + u) * 512 + lane * 16 + (it & 3) * 16384) & 65535);
+          if (kind == 3) {
+            st_shared_v4(addr, it, u, acc, 1u);
+          } else {
+            uint32_t x, y, z, q;
+            asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(x), "=r"(y), "=r"(z), "=r"(q) : "r"(addr));
+            acc += x ^ y ^ z ^ q;
+          }
+        }
+      } else if (kind == 5 || kind == 6) {
+        if (lane == 0) {
+          float* dst = mine + (it & 15) * 1024;
+          const uint32_t src = sX + w4 * 16384 + (it & 3) * 4096;
+          if (kind == 5)
+            asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], 4096;" ::"l"(dst), "r"(src)
+                         : "memory");
+          else
+            asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], 4096;" ::"l"(dst),
+                         "r"(src)
+                         : "memory");
+          bulk_commit();
+          asm volatile("cp.async.bulk.wait_group.read 4;" ::: "memory");
+        }
+        __syncwarp();
+      } else if (kind == 7) {
+        // rows of 128 floats: lanes with the same (lane & 3) cover 128 contiguous bytes of one row
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          float* pp = mine + (((it & 3) * 8 + u) * 4 + (lane & 3)) * 128 + (lane >> 2) * 4;
+          asm volatile("red.relaxed.gpu.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(pp), "f"(1.f), "f"(2.f),
+                       "f"(3.f), "f"(4.f)
+                       : "memory");
+        }
+      } else if (kind == 8) {
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          float x, y, z, q;
+          asm volatile("ld.global.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(x), "=f"(y), "=f"(z), "=f"(q)
+                       : "l"(mine + u * 128 + lane * 4));
+          acc += __float_as_uint(x) ^ __float_as_uint(q);
+        }
+      } else {
+        // 128 columns per lane; per 4 columns two butterfly stages (xor 2, xor 1) leave
+        // lane 4 k + j holding column j of its quad's 4 x 4 block, added as one vector
+        const int j = lane & 3;
+        const bool hi = (j & 2) != 0, odd = (j & 1) != 0;
+#pragma unroll 4
+        for (int c = 0; c < 128; c += 4) {
+          const float x0 = static_cast<float>(c + it), x1 = x0 + 1.f, x2 = x0 + 2.f, x3 = x0 + 3.f;
+          const float r0 = __shfl_xor_sync(0xffffffffu, hi ? x0 : x2, 2);
+          const float r1 = __shfl_xor_sync(0xffffffffu, hi ? x1 : x3, 2);
+          const float w0 = hi ? r0 : x0, w1 = hi ? r1 : x1, w2 = hi ? x2 : r0, w3 = hi ? x3 : r1;
+          const float q0 = __shfl_xor_sync(0xffffffffu, odd ? w0 : w1, 1);
+          const float q1 = __shfl_xor_sync(0xffffffffu, odd ? w2 : w3, 1);
+          float* pp = mine + (c + j) * 128 + 4 * (lane >> 2);
+          asm volatile("red.relaxed.gpu.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(pp),
+                       "f"(odd ? q0 : w0), "f"(odd ? w1 : q0), "f"(odd ? q1 : w2), "f"(odd ? w3 : q1)
+                       : "memory");
+        }
+      }
+    }
+    if ((kind == 5 || kind == 6) && lane == 0) bulk_wait_all();
+    if (lane == 0) atomicAdd(ops + blockIdx.x, n + (acc == 0xdeadbeefu ? 1u : 0u));
+  }
+  if (tid == 0) {
+    const uint64_t t0 = globaltimer_ns();
+    bool done = false;
+    while (!(done = mbar_try_wait(&bar, 0)) && globaltimer_ns() - t0 < 2000000000ull) {
+    }
+    if (!done) atomicExch(status, 1);
+    cycles[blockIdx.x] = clock64() - c0;
+    stop = 1;
+  }
+  __syncwarp();
+  tc_fence_before();
+  if (MODE == 2) cluster_sync_all(); else __syncthreads();
+  tc_fence_after();
+  if (warp == 0) {
+    if (MODE == 2)
+      asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, 512;" ::"r"(tmem) : "memory");
+    else
+      tmem_dealloc(tmem, 512);
+  }
+}
+
+cudaError_t launch_mma_rate(int mode, int N, int kind, int grid, int reps, unsigned long long* cycles,
+                            unsigned long long* ops, float* scratch, int* status, cudaStream_t s) {
+  auto go = [&](auto kernel) -> cudaError_t {
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kRateSmem);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid));
+    cfg.blockDim = dim3(256);
+    cfg.dynamicSmemBytes = kRateSmem;
+    cfg.stream = s;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = (mode == 2) ? 2 : 1;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, N, reps, kind, cycles, ops, scratch, status);
+  };
+  if (mode == 0) return go(mma_rate_kernel<0>);
+  if (mode == 1) return go(mma_rate_kernel<1>);
+  return go(mma_rate_kernel<2>);
+}
+
 // The current device must be an sm_100 part (tcgen05).
 int probe_device_ok() {
   int dev = 0, major = 0, minor = 0;
@@ -425,6 +651,20 @@ int fa_debug_umma_2cta(const void* A, const void* B, float* D, int N, int K, int
   if (rc != FA_OK) return rc;
   const cudaError_t e = fa::launch_umma2_probe(A, B, D, N, K, b_mn_major ? 1 : 0, a_tmem ? 1 : 0, status,
                                                static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
+}
+
+int fa_debug_mma_rate(int mode, int n, int kind, int grid, int reps, unsigned long long* cycles,
+                      unsigned long long* ops, float* scratch, int* status, void* stream) {
+  if (!cycles || !ops || !scratch || !status) return FA_ERR_INVALID_ARG;
+  if (mode < 0 || mode > 2 || kind < 0 || kind > 9 || grid < 1 || grid > 4096 || reps < 1 || reps > 100000)
+    return FA_ERR_INVALID_ARG;
+  if (mode == 2 ? (n != 128 && n != 256) || grid % 2 != 0 : (n != 64 && n != 128 && n != 256))
+    return FA_ERR_UNSUPPORTED;
+  const int rc = fa::probe_device_ok();
+  if (rc != FA_OK) return rc;
+  const cudaError_t e = fa::launch_mma_rate(mode, n, kind, grid, reps, cycles, ops, scratch, status,
+                                            static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
 }
 

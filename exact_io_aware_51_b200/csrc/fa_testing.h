@@ -30,6 +30,20 @@
  *     B's rows [r N / 2, (r + 1) N / 2) (K-major, or N-contiguous with
  *     b_mn_major).  N = 128, K = 64 or 128.  *status (device int) is set to 1
  *     if the MMAs did not complete within 2 s.
+ *   fa_debug_mma_rate: tensor-pipe rate.  `grid` CTAs (mode 2: grid / 2 CTA
+ *     pairs), one per SM, each issue reps x 8 back-to-back 128 x n x 16 bf16
+ *     MMAs into one TMEM accumulator (mode 0: both operands in shared memory;
+ *     1: A in tensor memory; 2: M = 256 over a CTA pair with cta_group::2,
+ *     n = 128 or 256) and write the SM clocks until completion to
+ *     cycles[grid].  With kind > 0 four more warps per CTA load the SM with
+ *     one kind of traffic (1 tcgen05.ld, 2 tcgen05.st, 3 st.shared,
+ *     4 ld.shared, 5 bulk copy shared -> global, 6 bulk fp32 reduce-add,
+ *     7 red.global.add.v4.f32, 8 ld.global hitting L1, 9 a quad transpose
+ *     then red.global.add.v4.f32) and add their operation count to
+ *     ops[grid] (4 KB per operation, 16 KB for kind 9).  scratch: device
+ *     floats, grid x 4 x 16384 of them.  cycles and ops: device arrays of
+ *     64-bit counters (ops zeroed by the caller).  *status set to 1 if the
+ *     MMAs did not complete within 2 s.
  * Return values are the fa_status codes of include/fa.h.
  */
 #ifndef FA_TESTING_H
@@ -46,6 +60,8 @@ int fa_debug_umma(const void* A, const void* B, float* D, int N, int K, int a_mn
 int fa_debug_umma_f8(const void* A, const void* B, float* D, int N, int b_mn_major, int a_tmem, void* stream);
 int fa_debug_umma_2cta(const void* A, const void* B, float* D, int N, int K, int b_mn_major, int a_tmem, int* status,
                        void* stream);
+int fa_debug_mma_rate(int mode, int n, int kind, int grid, int reps, unsigned long long* cycles,
+                      unsigned long long* ops, float* scratch, int* status, void* stream);
 
 #ifdef __cplusplus
 }

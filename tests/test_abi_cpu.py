@@ -62,6 +62,13 @@ def test_test_only_symbols_live_outside_the_public_header(L):
             assert name in exported, (lib_name, name)
     probe = fa.probe_lib()
     assert probe.fa_debug_umma(None, None, None, 64, 64, 0, 0, 0, None) == -1
+    # the rate probe validates before touching a device: null buffers, bad shapes, odd pair grids
+    assert probe.fa_debug_mma_rate(0, 128, 0, 148, 10, None, None, None, None, None) == -1
+    fake = 1 << 20  # never dereferenced: the checks fail first
+    assert probe.fa_debug_mma_rate(0, 96, 0, 148, 10, fake, fake, fake, fake, None) == -2
+    assert probe.fa_debug_mma_rate(2, 64, 0, 148, 10, fake, fake, fake, fake, None) == -2
+    assert probe.fa_debug_mma_rate(2, 128, 0, 147, 10, fake, fake, fake, fake, None) == -2
+    assert probe.fa_debug_mma_rate(0, 128, 10, 148, 10, fake, fake, fake, fake, None) == -1
 
 
 def test_checking_build_exports_the_same_symbols(L):

@@ -82,3 +82,39 @@ def test_umma_tile_two_cta(k, b_mn, a_tmem):
     torch.cuda.synchronize()
     ref = a.double().numpy() @ b.double().numpy().T
     assert rel_err(d.cpu(), ref) < 1e-5
+
+
+# Tensor-pipe rate (mode, n, traffic kind): the bare pipe for each MMA form the kernels
+# could use, then a 128 x 128 x 16 stream under each kind of concurrent traffic.
+RATE_CASES = ([(0, n, 0) for n in (64, 128, 256)] + [(1, n, 0) for n in (64, 128, 256)]
+              + [(2, n, 0) for n in (128, 256)]
+              + [(0, 128, k) for k in range(1, 10)] + [(1, 128, k) for k in (3, 4, 5, 6, 9)])
+
+
+@pytest.mark.gpu
+def test_mma_rate_table():
+    """Clocks per MMA on every SM at once, and what concurrent traffic gets.
+
+    Pins what the kernels' design rests on: a 128 x 128 x 16 MMA takes about 64
+    SM clocks whether B alone or both operands come from shared memory, N = 256 and
+    the CTA pair give no more per SM, N = 64 costs more per unit of work, and while
+    MMAs with both operands in shared memory run, shared-memory reads by the LSU
+    and by bulk copies are starved while stores, TMEM traffic and L1 loads are not.
+    `-s` prints the table (one JSON line per case)."""
+    need_gpu()
+    import json
+    rows = {}
+    for mode, n, kind in RATE_CASES:
+        r = fa.debug_mma_rate(mode, n, kind)
+        rows[(mode, n, kind)] = r
+        print(json.dumps(r))
+    unit = lambda m, n, k=0: rows[(m, n, k)]["clk_per_128x128x16"]
+    traffic = lambda m, k: rows[(m, 128, k)]["traffic_bytes_per_clk"]
+    for m, n in ((0, 128), (0, 256), (1, 128), (1, 256), (2, 128), (2, 256)):
+        assert unit(m, n) < 72.0, (m, n, unit(m, n))
+    assert unit(0, 64) > 1.2 * unit(0, 128)
+    for k in (1, 2, 3, 8):  # TMEM loads / stores, shared stores, L1 loads: the MMAs keep their rate
+        assert unit(0, 128, k) < 72.0, (k, unit(0, 128, k))
+    # shared-memory reads next to MMAs reading both operands from shared memory vs. B only
+    assert traffic(0, 4) < 0.5 * traffic(1, 4), (traffic(0, 4), traffic(1, 4))
+    assert traffic(0, 6) < 0.5 * traffic(1, 6), (traffic(0, 6), traffic(1, 6))
