@@ -37,7 +37,10 @@
 //     once its last S MMA is done) in the 128-byte swizzled layout and written
 //     by TMA tile stores (whole coalesced lines); LSE = (m + log2 l) ln 2.
 // The two query tiles ping-pong: while the softmax of one tile runs, the
-// tensor pipe computes the other tile's products.
+// tensor pipe computes the other tile's products.  Short walks (a query row
+// sees at most 768 keys) run one query tile per CTA and two CTAs per SM
+// instead (half the tensor memory, under half the shared memory each), which
+// ping-pong the same way and overlap each other's start and end.
 #include <cuda_bf16.h>
 
 #include "fa_internal.h"
@@ -48,12 +51,23 @@ namespace {
 
 constexpr int kBM = 128;        // query rows per tile = TMEM lanes
 constexpr int kBN = 128;        // keys per K/V tile
-constexpr int kThreads = 384;   // WG0, WG1: softmax; WG2: loader warp, MMA warp, 2 spare
-// Register split (per thread): 384 x 168 at launch = 256 x 216 + 128 x 72.
-constexpr uint32_t kRegSoftmax = 216;
-constexpr uint32_t kRegOther = 72;
-static_assert(kRegSoftmax >= 168 && kRegOther <= 168, "setmaxnreg direction (launch count 168)");
-static_assert(2 * kRegSoftmax + kRegOther == 3 * 168, "register split must match the launch");
+// kT query tiles per CTA: 2 (one CTA per SM) or 1 (two CTAs per SM, each with
+// half the tensor memory and under half the shared memory).  Warpgroups: kT
+// softmax warpgroups, then one with the loader warp, the MMA warp and 2 spare.
+template <int kT>
+struct FwdShape {
+  static constexpr int kThreads = 128 * (kT + 1);
+  static constexpr int kMinBlocks = (kT == 1) ? 2 : 1;
+  // Register split (per thread): kT = 2: 384 x 168 at launch = 256 x 216 + 128 x 72;
+  // kT = 1: 256 x 128 = 128 x 192 + 128 x 64 (two CTAs share the register file).
+  static constexpr uint32_t kRegLaunch = (kT == 1) ? 128 : 168;
+  static constexpr uint32_t kRegSoftmax = (kT == 1) ? 192 : 216;
+  static constexpr uint32_t kRegOther = (kT == 1) ? 64 : 72;
+  static constexpr uint32_t kTmemCols = (kT == 1) ? 256 : 512;
+  static_assert(kRegSoftmax >= kRegLaunch && kRegOther <= kRegLaunch, "setmaxnreg direction");
+  static_assert(kT * kRegSoftmax + kRegOther == (kT + 1) * kRegLaunch, "register split must match the launch");
+  static_assert(kThreads * kRegLaunch * kMinBlocks <= 65536, "register file");
+};
 // Lazy-rescale threshold (log2 units).  A stale m leaves every p <= 2^kTau, so
 // l <= 2^kTau * N and |O| <= 2^kTau * N * max|V| stay far inside fp32 for any
 // N < 2^31; bf16 P keeps its relative precision at any scale.  12 rather than
@@ -67,14 +81,15 @@ constexpr float kTau = 12.0f;
 // were 6-10% slower than none), so it is off.
 constexpr int kPolyEvery = 0;
 
-template <int D>
+template <int D, int kT>
 struct FwdCfg {
   static constexpr int kSub = D / 64;                 // 64-feature sub-tiles per row
   static constexpr int kSubBytes = kBM * 128;         // one [128][64] bf16 sub-tile
   static constexpr int kTileBytes = kSub * kSubBytes; // one 128 x D tile
-  static constexpr int kStages = (D == 128) ? 2 : 4;
+  // K/V ring depth: two CTAs per SM (kT = 1) keep half as many stages each
+  static constexpr int kStages = ((D == 128) ? 2 : 4) / (3 - kT);
   static constexpr int kOffQ = 0;
-  static constexpr int kOffK = 2 * kTileBytes;
+  static constexpr int kOffK = kT * kTileBytes;
   static constexpr int kOffV = kOffK + kStages * kTileBytes;
   static constexpr int kOffBar = kOffV + kStages * kTileBytes;
   static constexpr int kOffList = kOffBar + 512;           // block-sparse: the CTA's key-tile list
@@ -82,7 +97,7 @@ struct FwdCfg {
   static constexpr int kSmemBytesSparse = kOffList + 4 * kMaxSparseTiles + 1024;
   // TMEM columns: S_0 | S_1 | O_0 | O_1
   __device__ static constexpr uint32_t colS(int t) { return static_cast<uint32_t>(t) * 128u; }
-  __device__ static constexpr uint32_t colO(int t) { return 256u + static_cast<uint32_t>(t) * D; }
+  __device__ static constexpr uint32_t colO(int t) { return kT * 128u + static_cast<uint32_t>(t) * D; }
   static constexpr uint32_t kIdescS = idesc_bf16(kBM, kBN, 0, 0);
   static constexpr uint32_t kIdescPV = idesc_bf16(kBM, D, 0, 1);
 };
@@ -99,12 +114,16 @@ struct FwdBars {
 
 __device__ __forceinline__ bool warp_all(bool ok) { return __all_sync(0xffffffffu, ok); }
 
-template <int D, bool kSparse>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int D, bool kSparse, int kT>
+__global__ void __launch_bounds__(FwdShape<kT>::kThreads, FwdShape<kT>::kMinBlocks)
     fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO, const FwdArgs a,
                     const DevCtl ctl) {
-  using C = FwdCfg<D>;
+  using C = FwdCfg<D, kT>;
+  using W = FwdShape<kT>;
+  static_assert(kT == 2 || !kSparse, "block-sparse walks pair two query tiles");
+  constexpr int kThreads = W::kThreads;
+  constexpr int kLoaderWarp = 4 * kT, kMmaWarp = 4 * kT + 1;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   FwdBars* bars = reinterpret_cast<FwdBars*>(smem + C::kOffBar);
@@ -131,10 +150,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   int q0[2], klo[2], nkt[2];
 #pragma unroll
   for (int t = 0; t < 2; ++t) {
-    q0[t] = cb * 2 * kBM + t * kBM;
+    q0[t] = cb * kT * kBM + t * kBM;
     klo[t] = 0;
     nkt[t] = 0;
-    if (q0[t] < a.N) {
+    if (t < kT && q0[t] < a.N) {
       const int qmax = min(q0[t] + kBM - 1, a.N - 1);
       klo[t] = max(0, q0[t] - a.wl) / kBN;
       nkt[t] = min(a.N - 1, qmax + a.wr) / kBN + 1 - klo[t];
@@ -212,14 +231,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     bars->abort = (*reinterpret_cast<volatile unsigned int*>(ctl.abort_epoch) == ctl.epoch) ? 1 : 0;
     fence_mbar_init();
   }
-  if (warp == 9) tmem_alloc(&bars->tmem_base, 512);
+  if (warp == kMmaWarp) tmem_alloc(&bars->tmem_base, W::kTmemCols);
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
   const WaitCtl w{&bars->abort, ctl.status, ctl.abort_epoch, ctl.epoch, ctl.limit_ns};
 
-  if (warp < 8) {
-    reg_alloc<kRegSoftmax>();
+  if (warp < 4 * kT) {
+    reg_alloc<W::kRegSoftmax>();
     if (bars->abort == 0) {
       // ===================== softmax warps =====================
       const int t = warp >> 2;
@@ -377,8 +396,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else {
-    reg_dealloc<kRegOther>();
-    if (bars->abort == 0 && warp == 8) {
+    reg_dealloc<W::kRegOther>();
+    if (bars->abort == 0 && warp == kLoaderWarp) {
       // ===================== TMA producer =====================
       if (lane == 0) {
         tma_prefetch_desc(&tmQ);
@@ -422,7 +441,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         drain_ring(bars->k_full, C::kStages, k_issued, ctl.limit_ns);
         drain_ring(bars->v_full, C::kStages, v_issued, ctl.limit_ns);
       }
-    } else if (warp == 9) {
+    } else if (warp == kMmaWarp) {
       // ===================== MMA issuer (one thread) =====================
       if (lane == 0) {
         const uint32_t sQ = smem_u32(smem + C::kOffQ);
@@ -498,30 +517,53 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // ---- teardown ----
   __syncthreads();
-  if (warp == 9) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    tmem_dealloc(tmem, W::kTmemCols);
   }
 }
 
 }  // namespace
 
+// One query tile per CTA (two CTAs per SM) when a query row sees 768 keys or
+// fewer on average (N <= 512, causal N <= 1536, short windows): there the
+// CTAs' prologues, first loads and epilogues weigh on the few key tiles each
+// CTA walks, and a second CTA on the SM overlaps them.  Longer walks keep two
+// tiles per CTA, which load each K/V tile once for both.  Measured on B200,
+// two tiles -> one tile per CTA: causal B4 H16 N1024 d64 0.035 -> 0.031 ms,
+// causal B8 H16 N1024 d128 0.071 -> 0.063, B16 H16 N512 d64 0.051 -> 0.047 and
+// causal 0.047 -> 0.040; but B4 H16 N1024 d64 0.042 -> 0.044, B4 H32 N2048
+// d128 0.267 -> 0.283 and B1 H32 N16384 d128 3.54 -> 4.19.
+bool one_tile_per_cta(const FwdArgs& a) {
+  const long long n = a.N;
+  const long long left = (a.wl >= a.N) ? n - 1 : a.wl;
+  const long long right = (a.wr >= a.N) ? n - 1 : a.wr;
+  // keys per query row, ignoring the sequence edges (causal: half the sequence on average)
+  const long long seen = a.causal ? (n + 1) / 2 : ((left + right + 1 < n) ? left + right + 1 : n);
+  return seen <= 768;
+}
+
 cudaError_t launch_fwd_bf16(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& to,
                             const FwdArgs& a, const DevCtl& c, cudaStream_t s) {
-  const int nqb = (a.N + 2 * kBM - 1) / (2 * kBM);
-  const dim3 grid(nqb, a.H, a.B);
-  auto run = [&](auto kernel, int smem) -> cudaError_t {
+  const bool sparse = a.block_mask != nullptr;
+  const bool one = !sparse && one_tile_per_cta(a);
+  const int rows = (one ? 1 : 2) * kBM;
+  const dim3 grid((a.N + rows - 1) / rows, a.H, a.B);
+  auto run = [&](auto kernel, int smem, int threads) -> cudaError_t {
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    kernel<<<grid, kThreads, smem, s>>>(tq, tk, tv, to, a, c);
+    kernel<<<grid, threads, smem, s>>>(tq, tk, tv, to, a, c);
     return cudaGetLastError();
   };
-  const bool sparse = a.block_mask != nullptr;
-  if (a.d == 128)
-    return sparse ? run(fwd_bf16_kernel<128, true>, FwdCfg<128>::kSmemBytesSparse)
-                  : run(fwd_bf16_kernel<128, false>, FwdCfg<128>::kSmemBytes);
-  return sparse ? run(fwd_bf16_kernel<64, true>, FwdCfg<64>::kSmemBytesSparse)
-                : run(fwd_bf16_kernel<64, false>, FwdCfg<64>::kSmemBytes);
+  constexpr int k1 = FwdShape<1>::kThreads, k2 = FwdShape<2>::kThreads;
+  if (a.d == 128) {
+    if (sparse) return run(fwd_bf16_kernel<128, true, 2>, FwdCfg<128, 2>::kSmemBytesSparse, k2);
+    return one ? run(fwd_bf16_kernel<128, false, 1>, FwdCfg<128, 1>::kSmemBytes, k1)
+               : run(fwd_bf16_kernel<128, false, 2>, FwdCfg<128, 2>::kSmemBytes, k2);
+  }
+  if (sparse) return run(fwd_bf16_kernel<64, true, 2>, FwdCfg<64, 2>::kSmemBytesSparse, k2);
+  return one ? run(fwd_bf16_kernel<64, false, 1>, FwdCfg<64, 1>::kSmemBytes, k1)
+             : run(fwd_bf16_kernel<64, false, 2>, FwdCfg<64, 2>::kSmemBytes, k2);
 }
 
 }  // namespace fa
