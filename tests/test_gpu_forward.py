@@ -188,3 +188,27 @@ def test_bf16_n16k_kspike_forward_sampled_rows(causal):
     need_gpu()
     q, k, v, _ = I.workload_inputs(I.BF16_FWDBWD_N16K, with_do=False)
     _check_sampled(q, k, v, causal, [(0, 0), (0, 13), (0, 31)], nrows=512)
+
+
+# The bf16 forward takes one query tile per CTA (two CTAs per SM) when a query row
+# sees at most 768 keys on average, two tiles per CTA otherwise.  Each case sits on
+# one side of that rule: non-causal N = 768 / 769, causal N = 1535 / 1536, and a
+# window of 767 keys on a longer sequence (one tile) against 769 (two).
+@pytest.mark.gpu
+@pytest.mark.parametrize("n,causal,window", [(768, False, None), (769, False, None), (1535, True, None),
+                                             (1536, True, None), (2000, False, (700, 66)),
+                                             (2000, False, (700, 68))],
+                         ids=["n768", "n769", "causal1535", "causal1536", "window767", "window769"])
+@pytest.mark.parametrize("d", [64, 128])
+def test_bf16_one_and_two_tiles_per_cta(n, causal, window, d):
+    need_gpu()
+    q, k, v, _ = I.make_inputs(1, n, 3, d, seed=n + d, with_do=False, kv_heads=1)
+    sc = _scale(d)
+    kw = {"window": window} if window else {"causal": causal}
+    o, lse = fa.fwd(q.cuda(), k.cuda(), v.cuda(), scale=sc, **kw)
+    torch.cuda.synchronize()
+    assert fa.last_device_status()[0] == 0
+    o_ref, l_ref = oracle.forward(q, k, v, sc, causal, **({"window": window} if window else {}))
+    assert np.isfinite(f64(o)).all()
+    assert rel_err(o.cpu(), o_ref) <= TOL_BF16_REL
+    assert abs_err(lse.cpu(), l_ref) <= TOL_LSE
