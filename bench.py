@@ -499,18 +499,25 @@ def run_ours(args, world, rank, local):
             fa.fwd_fp8(*codes, *scales, causal=causal, scale=scale, out=o8, lse=lse)
         n8 = max(3, min(args.steps, 10))
         e8a, e8b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        clk8 = NvmlSampler(local)  # the leg follows the power-capped region: record its own clock
+        clk8.start()
         barrier()
         torch.cuda.synchronize()
+        clk8.mark_begin()
         e8a.record(stream)
         for _ in range(n8):
             fa.fwd_fp8(*codes, *scales, causal=causal, scale=scale, out=o8, lse=lse)
         e8b.record(stream)
         torch.cuda.synchronize()
+        clk8.mark_end()
         barrier()
+        c8 = clk8.stop()
         ms8 = slowest(e8a.elapsed_time(e8b)) / n8
         tf8 = f / (ms8 * 1e-3) / 1e12
         fp8 = {"tflops": tf8, "ms": ms8, "launches": n8, "peak": 2 * peak_burst,
                "frac_of_peak": tf8 / (2 * peak_burst),
+               "frac_at_max_clock": clock_scaled(tf8 / (2 * peak_burst), c8),
+               "sm_mhz": (c8 or {}).get("sm_mhz"), "reasons": (c8 or {}).get("reasons"),
                "peak_source": "bf16 burst x 2 (the nominal e4m3 / bf16 dense ratio)",
                "inputs": "Q, K, V of the same workload as e4m3 codes with per-tensor scales"}
         del codes, o8
