@@ -474,7 +474,9 @@ def debug_umma_2cta(a: torch.Tensor, b: torch.Tensor, b_mn_major: int, a_tmem: i
 
 
 MMA_RATE_KINDS = ("none", "tcgen05.ld", "tcgen05.st", "st.shared", "ld.shared", "bulk copy smem->global",
-                  "bulk reduce-add smem->global", "red.global.add.v4", "ld.global (L1)", "quad transpose + red.v4")
+                  "bulk reduce-add smem->global", "red.global.add.v4", "ld.global (L1)", "quad transpose + red.v4",
+                  "FFMA-bound warp on every SMSP", "FFMA-bound warp on the issuer's SMSP only",
+                  "FFMA-bound warps on the other SMSPs only", "FFMA-bound warp on every SMSP, two issuers")
 
 
 def debug_mma_rate(mode: int, n: int, kind: int = 0, grid: int | None = None, reps: int = 1500, device=None) -> dict:
@@ -504,7 +506,7 @@ def debug_mma_rate(mode: int, n: int, kind: int = 0, grid: int | None = None, re
     ctas = 2 if mode == 2 else 1
     return {"mode": mode, "n": n, "kind": MMA_RATE_KINDS[kind], "grid": grid, "clk_per_mma": per,
             "clk_per_128x128x16": per * (128 * 128) / (m // ctas * n),
-            "traffic_bytes_per_clk": o * (16384.0 if kind == 9 else 4096.0) / c if kind else 0.0}
+            "traffic_bytes_per_clk": o * (16384.0 if kind == 9 else 4096.0) / c if 0 < kind < 10 else 0.0}
 
 
 class _Attention(torch.autograd.Function):

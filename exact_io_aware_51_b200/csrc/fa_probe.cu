@@ -390,7 +390,11 @@ cudaError_t launch_umma2_probe(const void* A, const void* B, float* D, int N, in
 //   1 tcgen05.ld, 2 tcgen05.st (TMEM columns 256-383), 3 st.shared,
 //   4 ld.shared, 5 bulk copy shared -> global, 6 bulk fp32 reduce-add
 //   shared -> global, 7 red.global.add.v4.f32 from registers, 8 ld.global
-//   (L1 hits), 9 a 4 x 4 transpose in lane quads then red.global.add.v4.f32.
+//   (L1 hits), 9 a 4 x 4 transpose in lane quads then red.global.add.v4.f32,
+//   10 FFMA-bound code on warps 4-7 (one per SMSP), 11 the same on warp 4
+//   only (the issuer's SMSP), 12 on warps 5-7 only (the other SMSPs), 13 as
+//   10 with the MMAs split over two issuers (warps 0 and 1, SMSPs 0 and 1,
+//   each into its own accumulator).
 // Operand values are arbitrary: only the timing is read.
 // ---------------------------------------------------------------------------
 constexpr int kRateSmem = 200 * 1024;  // more than half the SM's shared memory: one CTA per SM
@@ -404,7 +408,7 @@ __global__ void __launch_bounds__(256, 1)
   const uint32_t sA = smem_u32(smem);              // [128][128] bf16, two 16 KB K-chunks
   const uint32_t sB = smem_u32(smem + 32768);      // up to [256][128] bf16, two K-chunks
   const uint32_t sX = smem_u32(smem + 98304);      // 64 KB the traffic warps read and write
-  __shared__ uint64_t bar;
+  __shared__ uint64_t bar, bar2;
   __shared__ uint32_t tbase;
   __shared__ volatile int stop;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -413,6 +417,7 @@ __global__ void __launch_bounds__(256, 1)
   if (tid == 0) {
     stop = 0;
     mbar_init(&bar, 1);
+    mbar_init(&bar2, 1);
     fence_mbar_init();
   }
   if (warp == 0) {
@@ -440,28 +445,47 @@ __global__ void __launch_bounds__(256, 1)
   if (MODE == 2) cluster_sync_all(); else __syncthreads();
   tc_fence_after();
 
-  const bool issuer = tid == 0 && (MODE != 2 || cluster_rank() == 0);
+  const bool two = kind == 13;  // a second issuer: lane 0 of warp 1, its own accumulator at column 128
+  const bool issuer = (tid == 0 && (MODE != 2 || cluster_rank() == 0)) || (two && tid == 32);
   const unsigned long long c0 = clock64();
   if (issuer) {
     const int nb = (MODE == 2) ? N / 2 : N;  // B rows in this CTA
     const uint32_t idesc = (MODE == 1) ? idesc_bf16(128, N, 0, 1) : idesc_bf16(MODE == 2 ? 256 : 128, N, 0, 0);
-    for (int r = 0; r < reps; ++r) {
+    if (!two) {
+      // the plain stream: nothing between the MMAs but their constant offsets
+      for (int r = 0; r < reps; ++r) {
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        const uint32_t acc = (r > 0 || kk > 0) ? 1u : 0u;
-        const uint64_t ad = sw128_desc(sA + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-        const uint64_t bd = sw128_desc(sB + (kk >> 2) * (nb * 128) + (kk & 3) * 32, 16, 1024);
-        if (MODE == 0) {
-          umma_ss(tmem, ad, bd, idesc, acc);
-        } else if (MODE == 1) {
-          // B MN-major: 16 K-rows of 128 bytes per step, N groups of 64 at 16 KB
-          umma_ts(tmem, tmem + 384 + kk * 8, sw128_desc(sB + kk * 2048, 16384, 1024), idesc, acc);
-        } else {
-          asm volatile(
-              "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-              "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem),
-              "l"(ad), "l"(bd), "r"(idesc), "r"(acc)
-              : "memory");
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t acc = (r > 0 || kk > 0) ? 1u : 0u;
+          const uint64_t ad = sw128_desc(sA + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+          const uint64_t bd = sw128_desc(sB + (kk >> 2) * (nb * 128) + (kk & 3) * 32, 16, 1024);
+          if (MODE == 0) {
+            umma_ss(tmem, ad, bd, idesc, acc);
+          } else if (MODE == 1) {
+            // B MN-major: 16 K-rows of 128 bytes per step, N groups of 64 at 16 KB
+            umma_ts(tmem, tmem + 384 + kk * 8, sw128_desc(sB + kk * 2048, 16384, 1024), idesc, acc);
+          } else {
+            asm volatile(
+                "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem),
+                "l"(ad), "l"(bd), "r"(idesc), "r"(acc)
+                : "memory");
+          }
+        }
+      }
+    } else {
+      // two issuers (modes 0 and 1): half the groups each, each into its own accumulator
+      const uint32_t d = tmem + ((tid == 32) ? 128u : 0u);
+      const int my_reps = (tid == 32) ? reps - reps / 2 : reps / 2;
+      for (int r = 0; r < my_reps; ++r) {
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t acc = (r > 0 || kk > 0) ? 1u : 0u;
+          if (MODE == 1)
+            umma_ts(d, tmem + 384 + kk * 8, sw128_desc(sB + kk * 2048, 16384, 1024), idesc, acc);
+          else
+            umma_ss(d, sw128_desc(sA + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                    sw128_desc(sB + (kk >> 2) * (nb * 128) + (kk & 3) * 32, 16, 1024), idesc, acc);
         }
       }
     }
@@ -473,10 +497,30 @@ __global__ void __launch_bounds__(256, 1)
           "h"(mask)
           : "memory");
     } else {
-      umma_commit(&bar);
+      umma_commit(tid == 32 ? &bar2 : &bar);
     }
   }
-  if (warp >= 4 && kind > 0) {
+  if (kind >= 10) {
+    // FFMA-bound warps: eight independent chains, so every cycle has an instruction ready
+    const bool busy = (kind == 11) ? warp == 4 : (kind == 12) ? (warp >= 5 && warp <= 7) : (warp >= 4 && warp <= 7);
+    if (busy) {
+      float f[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) f[i] = static_cast<float>(lane + i);
+      unsigned long long n = 0;
+      for (int it = 0; it < 1000000 && !stop; ++it, ++n) {
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) f[i] = fmaf(f[i], 0.999f, 0.5f);
+        }
+      }
+      float sum = 0.f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) sum += f[i];
+      if (lane == 0) atomicAdd(ops + blockIdx.x, n + (sum == 12345.f ? 1u : 0u));
+    }
+  } else if (warp >= 4 && kind > 0) {
     const int w4 = warp - 4;
     const uint32_t lane_bits = static_cast<uint32_t>(w4 * 32) << 16;
     float* mine = scratch + (static_cast<size_t>(blockIdx.x) * 4 + w4) * 16384;  // this warp's 64 KB
@@ -566,6 +610,10 @@ __global__ void __launch_bounds__(256, 1)
     const uint64_t t0 = globaltimer_ns();
     bool done = false;
     while (!(done = mbar_try_wait(&bar, 0)) && globaltimer_ns() - t0 < 2000000000ull) {
+    }
+    if (done && two) {
+      while (!(done = mbar_try_wait(&bar2, 0)) && globaltimer_ns() - t0 < 2000000000ull) {
+      }
     }
     if (!done) atomicExch(status, 1);
     cycles[blockIdx.x] = clock64() - c0;
@@ -657,8 +705,9 @@ int fa_debug_umma_2cta(const void* A, const void* B, float* D, int N, int K, int
 int fa_debug_mma_rate(int mode, int n, int kind, int grid, int reps, unsigned long long* cycles,
                       unsigned long long* ops, float* scratch, int* status, void* stream) {
   if (!cycles || !ops || !scratch || !status) return FA_ERR_INVALID_ARG;
-  if (mode < 0 || mode > 2 || kind < 0 || kind > 9 || grid < 1 || grid > 4096 || reps < 1 || reps > 100000)
+  if (mode < 0 || mode > 2 || kind < 0 || kind > 13 || grid < 1 || grid > 4096 || reps < 1 || reps > 100000)
     return FA_ERR_INVALID_ARG;
+  if (kind == 13 && (mode == 2 || n > 128)) return FA_ERR_UNSUPPORTED;  // the second accumulator sits at column 128
   if (mode == 2 ? (n != 128 && n != 256) || grid % 2 != 0 : (n != 64 && n != 128 && n != 256))
     return FA_ERR_UNSUPPORTED;
   const int rc = fa::probe_device_ok();

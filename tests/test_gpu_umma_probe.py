@@ -88,7 +88,7 @@ def test_umma_tile_two_cta(k, b_mn, a_tmem):
 # could use, then a 128 x 128 x 16 stream under each kind of concurrent traffic.
 RATE_CASES = ([(0, n, 0) for n in (64, 128, 256)] + [(1, n, 0) for n in (64, 128, 256)]
               + [(2, n, 0) for n in (128, 256)]
-              + [(0, 128, k) for k in range(1, 10)] + [(1, 128, k) for k in (3, 4, 5, 6, 9)])
+              + [(0, 128, k) for k in range(1, 14)] + [(1, 128, k) for k in (3, 4, 5, 6, 9)])
 
 
 @pytest.mark.gpu
@@ -100,6 +100,8 @@ def test_mma_rate_table():
     the CTA pair give no more per SM, N = 64 costs more per unit of work, and while
     MMAs with both operands in shared memory run, shared-memory reads by the LSU
     and by bulk copies are starved while stores, TMEM traffic and L1 loads are not.
+    The issuing thread competes for its SMSP's issue slots: ALU-bound warps there
+    (not elsewhere) slow the MMA stream, and two issuers on two SMSPs recover it.
     `-s` prints the table (one JSON line per case)."""
     need_gpu()
     import json
@@ -118,3 +120,8 @@ def test_mma_rate_table():
     # shared-memory reads next to MMAs reading both operands from shared memory vs. B only
     assert traffic(0, 4) < 0.5 * traffic(1, 4), (traffic(0, 4), traffic(1, 4))
     assert traffic(0, 6) < 0.5 * traffic(1, 6), (traffic(0, 6), traffic(1, 6))
+    # issue slots: one ALU-bound warp on the issuing thread's SMSP slows the MMAs more than
+    # three on the other SMSPs, and a second issuer on another SMSP wins the rate back
+    assert unit(0, 128, 11) > 1.3 * unit(0, 128, 12), (unit(0, 128, 11), unit(0, 128, 12))
+    assert unit(0, 128, 12) < 72.0, unit(0, 128, 12)
+    assert unit(0, 128, 13) < 0.8 * unit(0, 128, 10), (unit(0, 128, 13), unit(0, 128, 10))
