@@ -476,7 +476,8 @@ def debug_umma_2cta(a: torch.Tensor, b: torch.Tensor, b_mn_major: int, a_tmem: i
 MMA_RATE_KINDS = ("none", "tcgen05.ld", "tcgen05.st", "st.shared", "ld.shared", "bulk copy smem->global",
                   "bulk reduce-add smem->global", "red.global.add.v4", "ld.global (L1)", "quad transpose + red.v4",
                   "FFMA-bound warp on every SMSP", "FFMA-bound warp on the issuer's SMSP only",
-                  "FFMA-bound warps on the other SMSPs only", "FFMA-bound warp on every SMSP, two issuers")
+                  "FFMA-bound warps on the other SMSPs only", "FFMA-bound warp on every SMSP, two issuers",
+                  "FFMA-bound warp on the issuer's SMSP, converged-warp issue")
 
 
 def debug_mma_rate(mode: int, n: int, kind: int = 0, grid: int | None = None, reps: int = 1500, device=None) -> dict:

@@ -13,7 +13,8 @@
 //   * one CTA owns two 128-row query tiles (t = 0, 1) of one (b, h) and
 //     streams 128-key K/V tiles through a TMA ring in shared memory
 //     (128-byte swizzle, mbarrier completion);
-//   * one thread issues all tcgen05 MMAs: S_t = Q_t K^T (both operands from
+//   * one warp issues all tcgen05 MMAs (converged, one lane elected per
+//     instruction): S_t = Q_t K^T (both operands from
 //     shared memory, accumulator in TMEM) and O_t += P_t V (P_t read straight
 //     from TMEM where the softmax wrote it over S_t, V from shared memory);
 //   * eight softmax warps (one TMEM lane = one query row per thread) read S_t,
@@ -442,8 +443,12 @@ __global__ void __launch_bounds__(FwdShape<kT>::kThreads, FwdShape<kT>::kMinBloc
         drain_ring(bars->v_full, C::kStages, v_issued, ctl.limit_ns);
       }
     } else if (warp == kMmaWarp) {
-      // ===================== MMA issuer (one thread) =====================
-      if (lane == 0) {
+      // ===================== MMA issuer (one warp) =====================
+      // The whole warp runs the loop (waits and descriptor arithmetic are
+      // warp-uniform) and one lane elected by elect.sync issues each MMA and
+      // commit: a lone lane-0 issuer loses its SMSP's issue slots to the
+      // ALU-bound softmax warps there and starves the tensor pipe.
+      {
         const uint32_t sQ = smem_u32(smem + C::kOffQ);
         const uint32_t sK = smem_u32(smem + C::kOffK);
         const uint32_t sV = smem_u32(smem + C::kOffV);
@@ -454,20 +459,20 @@ __global__ void __launch_bounds__(FwdShape<kT>::kThreads, FwdShape<kT>::kMinBloc
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t off = (kk >> 2) * C::kSubBytes + (kk & 3) * 32;
-            umma_ss(tmem + C::colS(t), sw128_desc(qa + off, 16, 1024), sw128_desc(kb + off, 16, 1024),
+            umma_ss_w(tmem + C::colS(t), sw128_desc(qa + off, 16, 1024), sw128_desc(kb + off, 16, 1024),
                     C::kIdescS, kk > 0 ? 1u : 0u);
           }
-          umma_commit(&bars->s_full[t]);
+          umma_commit_w(&bars->s_full[t]);
         };
         // O_t += P_t V_j (P_t from TMEM over S_t, V from ring stage s)
         auto issue_pv = [&](int t, int s, bool acc) {
           const uint32_t vb = sV + s * C::kTileBytes;
 #pragma unroll
           for (int kk = 0; kk < kBN / 16; ++kk) {
-            umma_ts(tmem + C::colO(t), tmem + C::colS(t) + kk * 8, sw128_desc(vb + kk * 2048, C::kSubBytes, 1024),
+            umma_ts_w(tmem + C::colO(t), tmem + C::colS(t) + kk * 8, sw128_desc(vb + kk * 2048, C::kSubBytes, 1024),
                     C::kIdescPV, (acc || kk > 0) ? 1u : 0u);
           }
-          umma_commit(&bars->o_done[t]);
+          umma_commit_w(&bars->o_done[t]);
         };
         // jl[t]: how many of query tile t's key tiles have had their P V issued
         int jl[2] = {0, 0};
@@ -476,28 +481,28 @@ __global__ void __launch_bounds__(FwdShape<kT>::kThreads, FwdShape<kT>::kMinBloc
         // pipe executes one thread's MMAs in issue order, so PV_t(j) has read
         // P_t(j) before S_t(j+1) writes there.  A query tile whose first key
         // tile is a later stream tile gets its first S in the iteration before.
-        bool ok = nk > 0 && wait_bar(&bars->q_full, 0, w, 3) && wait_bar(&bars->k_full[0], 0, w, 4);
+        bool ok = nk > 0 && warp_all(wait_bar(&bars->q_full, 0, w, 3)) && warp_all(wait_bar(&bars->k_full[0], 0, w, 4));
         if (ok) {
           tc_fence_after();
           for (int t = 0; t < 2; ++t)
             if (uses(t, 0)) issue_s(t, 0);
-          umma_commit(&bars->k_empty[0]);
+          umma_commit_w(&bars->k_empty[0]);
         }
         for (int j = 0; ok && j < nk; ++j) {
           const int s = j % C::kStages;
           const int sn = (j + 1) % C::kStages;
-          if (!(ok = wait_bar(&bars->v_full[s], (j / C::kStages) & 1, w, 6))) break;
+          if (!(ok = warp_all(wait_bar(&bars->v_full[s], (j / C::kStages) & 1, w, 6)))) break;
           bool next_k = false;
           for (int t = 0; t < 2; ++t) {
             if (uses(t, j)) {
-              if (!(ok = wait_bar(&bars->p_full[t], jl[t] & 1, w, 7))) break;
+              if (!(ok = warp_all(wait_bar(&bars->p_full[t], jl[t] & 1, w, 7)))) break;
               tc_fence_after();
               issue_pv(t, s, jl[t] > 0);
               ++jl[t];
             }
             if (j + 1 < nk && uses(t, j + 1)) {
               if (!next_k) {
-                if (!(ok = wait_bar(&bars->k_full[sn], ((j + 1) / C::kStages) & 1, w, 5))) break;
+                if (!(ok = warp_all(wait_bar(&bars->k_full[sn], ((j + 1) / C::kStages) & 1, w, 5)))) break;
                 tc_fence_after();
                 next_k = true;
               }
@@ -505,11 +510,11 @@ __global__ void __launch_bounds__(FwdShape<kT>::kThreads, FwdShape<kT>::kMinBloc
             }
           }
           if (!ok) break;
-          umma_commit(&bars->v_empty[s]);
-          if (next_k) umma_commit(&bars->k_empty[sn]);
+          umma_commit_w(&bars->v_empty[s]);
+          if (next_k) umma_commit_w(&bars->k_empty[sn]);
         }
         // all MMAs of this CTA finish before TMEM is released
-        umma_commit(&bars->drain);
+        umma_commit_w(&bars->drain);
         drain_wait(&bars->drain, 0, ctl.limit_ns);
       }
     }

@@ -394,7 +394,8 @@ cudaError_t launch_umma2_probe(const void* A, const void* B, float* D, int N, in
 //   10 FFMA-bound code on warps 4-7 (one per SMSP), 11 the same on warp 4
 //   only (the issuer's SMSP), 12 on warps 5-7 only (the other SMSPs), 13 as
 //   10 with the MMAs split over two issuers (warps 0 and 1, SMSPs 0 and 1,
-//   each into its own accumulator).
+//   each into its own accumulator), 14 as 11 with the MMAs issued by all of
+//   warp 0, converged, one lane elected by elect.sync (modes 0 and 1).
 // Operand values are arbitrary: only the timing is read.
 // ---------------------------------------------------------------------------
 constexpr int kRateSmem = 200 * 1024;  // more than half the SM's shared memory: one CTA per SM
@@ -446,9 +447,25 @@ __global__ void __launch_bounds__(256, 1)
   tc_fence_after();
 
   const bool two = kind == 13;  // a second issuer: lane 0 of warp 1, its own accumulator at column 128
+  const bool conv = kind == 14;  // all of warp 0 issues, converged, through elect.sync
   const bool issuer = (tid == 0 && (MODE != 2 || cluster_rank() == 0)) || (two && tid == 32);
   const unsigned long long c0 = clock64();
-  if (issuer) {
+  if (MODE != 2 && conv && warp == 0) {
+    const uint32_t idesc = (MODE == 1) ? idesc_bf16(128, N, 0, 1) : idesc_bf16(128, N, 0, 0);
+    for (int r = 0; r < reps; ++r) {
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t acc = (r > 0 || kk > 0) ? 1u : 0u;
+        if (MODE == 1)
+          umma_ts_w(tmem, tmem + 384 + kk * 8, sw128_desc(sB + kk * 2048, 16384, 1024), idesc, acc);
+        else
+          umma_ss_w(tmem, sw128_desc(sA + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                    sw128_desc(sB + (kk >> 2) * (N * 128) + (kk & 3) * 32, 16, 1024), idesc, acc);
+      }
+    }
+    umma_commit_w(&bar);
+    __syncwarp();
+  } else if (issuer && !conv) {
     const int nb = (MODE == 2) ? N / 2 : N;  // B rows in this CTA
     const uint32_t idesc = (MODE == 1) ? idesc_bf16(128, N, 0, 1) : idesc_bf16(MODE == 2 ? 256 : 128, N, 0, 0);
     if (!two) {
@@ -502,7 +519,7 @@ __global__ void __launch_bounds__(256, 1)
   }
   if (kind >= 10) {
     // FFMA-bound warps: eight independent chains, so every cycle has an instruction ready
-    const bool busy = (kind == 11) ? warp == 4 : (kind == 12) ? (warp >= 5 && warp <= 7) : (warp >= 4 && warp <= 7);
+    const bool busy = (kind == 11 || kind == 14) ? warp == 4 : (kind == 12) ? (warp >= 5 && warp <= 7) : (warp >= 4 && warp <= 7);
     if (busy) {
       float f[8];
 #pragma unroll
@@ -705,9 +722,10 @@ int fa_debug_umma_2cta(const void* A, const void* B, float* D, int N, int K, int
 int fa_debug_mma_rate(int mode, int n, int kind, int grid, int reps, unsigned long long* cycles,
                       unsigned long long* ops, float* scratch, int* status, void* stream) {
   if (!cycles || !ops || !scratch || !status) return FA_ERR_INVALID_ARG;
-  if (mode < 0 || mode > 2 || kind < 0 || kind > 13 || grid < 1 || grid > 4096 || reps < 1 || reps > 100000)
+  if (mode < 0 || mode > 2 || kind < 0 || kind > 14 || grid < 1 || grid > 4096 || reps < 1 || reps > 100000)
     return FA_ERR_INVALID_ARG;
   if (kind == 13 && (mode == 2 || n > 128)) return FA_ERR_UNSUPPORTED;  // the second accumulator sits at column 128
+  if (kind == 14 && mode == 2) return FA_ERR_UNSUPPORTED;
   if (mode == 2 ? (n != 128 && n != 256) || grid % 2 != 0 : (n != 64 && n != 128 && n != 256))
     return FA_ERR_UNSUPPORTED;
   const int rc = fa::probe_device_ok();

@@ -43,7 +43,9 @@
  *     ops[grid] (4 KB per operation, 16 KB for kind 9).  Kinds 10-13 run
  *     FFMA-bound warps instead: 10 one on every SMSP, 11 one on the issuer's
  *     SMSP only, 12 three on the other SMSPs, 13 as 10 with the MMAs split
- *     over two issuing threads on two SMSPs (modes 0 and 1, n <= 128).  scratch: device
+ *     over two issuing threads on two SMSPs (modes 0 and 1, n <= 128), 14 as
+ *     11 with the MMAs issued by a converged warp, one lane elected by
+ *     elect.sync (modes 0 and 1).  scratch: device
  *     floats, grid x 4 x 16384 of them.  cycles and ops: device arrays of
  *     64-bit counters (ops zeroed by the caller).  *status set to 1 if the
  *     MMAs did not complete within 2 s.

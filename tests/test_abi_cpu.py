@@ -68,7 +68,8 @@ def test_test_only_symbols_live_outside_the_public_header(L):
     assert probe.fa_debug_mma_rate(0, 96, 0, 148, 10, fake, fake, fake, fake, None) == -2
     assert probe.fa_debug_mma_rate(2, 64, 0, 148, 10, fake, fake, fake, fake, None) == -2
     assert probe.fa_debug_mma_rate(2, 128, 0, 147, 10, fake, fake, fake, fake, None) == -2
-    assert probe.fa_debug_mma_rate(0, 128, 14, 148, 10, fake, fake, fake, fake, None) == -1
+    assert probe.fa_debug_mma_rate(0, 128, 15, 148, 10, fake, fake, fake, fake, None) == -1
+    assert probe.fa_debug_mma_rate(2, 128, 14, 148, 10, fake, fake, fake, fake, None) == -2
     assert probe.fa_debug_mma_rate(0, 256, 13, 148, 10, fake, fake, fake, fake, None) == -2
     assert probe.fa_debug_mma_rate(2, 128, 13, 148, 10, fake, fake, fake, fake, None) == -2
 

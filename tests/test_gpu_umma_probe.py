@@ -88,7 +88,7 @@ def test_umma_tile_two_cta(k, b_mn, a_tmem):
 # could use, then a 128 x 128 x 16 stream under each kind of concurrent traffic.
 RATE_CASES = ([(0, n, 0) for n in (64, 128, 256)] + [(1, n, 0) for n in (64, 128, 256)]
               + [(2, n, 0) for n in (128, 256)]
-              + [(0, 128, k) for k in range(1, 14)] + [(1, 128, k) for k in (3, 4, 5, 6, 9)])
+              + [(0, 128, k) for k in range(1, 15)] + [(1, 128, k) for k in (3, 4, 5, 6, 9)])
 
 
 @pytest.mark.gpu
@@ -101,7 +101,8 @@ def test_mma_rate_table():
     MMAs with both operands in shared memory run, shared-memory reads by the LSU
     and by bulk copies are starved while stores, TMEM traffic and L1 loads are not.
     The issuing thread competes for its SMSP's issue slots: ALU-bound warps there
-    (not elsewhere) slow the MMA stream, and two issuers on two SMSPs recover it.
+    (not elsewhere) slow the MMA stream; two issuers on two SMSPs, or one converged
+    warp issuing through elect.sync, recover it.
     `-s` prints the table (one JSON line per case)."""
     need_gpu()
     import json
@@ -125,3 +126,5 @@ def test_mma_rate_table():
     assert unit(0, 128, 11) > 1.3 * unit(0, 128, 12), (unit(0, 128, 11), unit(0, 128, 12))
     assert unit(0, 128, 12) < 72.0, unit(0, 128, 12)
     assert unit(0, 128, 13) < 0.8 * unit(0, 128, 10), (unit(0, 128, 13), unit(0, 128, 10))
+    # and a converged warp issuing through elect.sync keeps its slots where a lone lane does not
+    assert unit(0, 128, 14) < 0.8 * unit(0, 128, 11), (unit(0, 128, 14), unit(0, 128, 11))
