@@ -372,6 +372,7 @@ def run_sweep(fa, I, dev, stream, main, peak, nvml):
     out.append(entry(I.BF16_FWDBWD_N4K, True, True))
     out.append(entry(I.BF16_FWDBWD_N16K, True, True, tensors=main))
     out.append(entry(I.BF16_FWDBWD_N16K, False, False, tensors=main))
+    out.append(entry(I.BF16_FWDBWD_N16K_D64, False, True))  # the d = 64 backward kernel
     for w in I.SWEEP:
         out += [entry(w, c, False) for c in (False, True)]
     out += [entry(I.BF16_GQA_H64_KV8, c, True) for c in (False, True)]

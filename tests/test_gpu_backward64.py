@@ -83,3 +83,19 @@ def test_bwd64_blocksparse():
     q, k, v, do = I.make_inputs(1, n, 2, D, seed=12)
     got = _run(q, k, v, do, block_mask=torch.from_numpy(m).cuda())
     _check(got, oracle.backward(q, k, v, do, _scale(), False, block_mask=m))
+
+
+@pytest.mark.gpu
+def test_bwd64_b1_h32_n16384_heads():
+    """The bench sweep's d = 64 workload at full size: the whole problem on the GPU,
+    two whole heads (first and last) against the oracle."""
+    need_gpu()
+    q, k, v, do = I.workload_inputs(I.BF16_FWDBWD_N16K_D64)
+    dq, dk, dv = _run(q, k, v, do, causal=False)
+    sc = _scale()
+    f64 = lambda t: t.float().numpy().astype(np.float64)
+    for h in (0, 31):
+        rq, rk, rv, _ = oracle.backward_head(*(f64(t[0, :, h]) for t in (q, k, v, do)), sc, False)
+        for g, r, name in ((dq[0, :, h], rq, "dq"), (dk[0, :, h], rk, "dk"), (dv[0, :, h], rv, "dv")):
+            assert torch.isfinite(g.float()).all(), (h, name)
+            assert rel_err(g, r) <= TOL_BF16_REL, (h, name)
