@@ -684,20 +684,22 @@ PROFILE_WORKLOAD = dict(B=1, H=64, N=4096, d=128)
 def run_profile_case(args):
     """Small case for ncu section captures: 2 x (forward, backward) on B1 H64 N4096 d128
     (each tensor 64 MiB, so the five of them exceed the L2; < 1 GB on the device), then
-    2 x the 8-bit forward on the same Q, K, V."""
+    2 x the 8-bit forward on the same Q, K, V.  With --profile-d64: the same at d = 64
+    (32 MiB tensors, five of them still beyond the L2), without the 8-bit forward."""
     import torch
 
     import exact_io_aware_51_b200 as fa
     from exact_io_aware_51_b200 import inputs as I
-    w = PROFILE_WORKLOAD
+    w = dict(PROFILE_WORKLOAD, d=64) if args.profile_d64 else PROFILE_WORKLOAD
     q, k, v, do = (t.cuda() for t in I.make_inputs(w["B"], w["N"], w["H"], w["d"], seed=0))
     for causal in ((False, True) if args.profile_causal else (False,)):
         for _ in range(2):
             o, lse = fa.fwd(q, k, v, causal=causal)
             fa.bwd(q, k, v, o, do, lse, causal=causal)
-    q8, k8, v8 = (t.to(torch.float8_e4m3fn) for t in (q, k, v))
-    for _ in range(2):
-        fa.fwd_fp8(q8, k8, v8, 1.0, 1.0, 1.0)
+    if w["d"] == 128:
+        q8, k8, v8 = (t.to(torch.float8_e4m3fn) for t in (q, k, v))
+        for _ in range(2):
+            fa.fwd_fp8(q8, k8, v8, 1.0, 1.0, 1.0)
     torch.cuda.synchronize()
     rc, detail = fa.last_device_status()
     if rc != 0:
@@ -735,6 +737,8 @@ def main():
     ap.add_argument("--profile-case", action="store_true",
                     help="run only the small profiling case (2 x fwd + bwd, B1 H64 N4096 d128) for ncu")
     ap.add_argument("--profile-causal", action="store_true", help="with --profile-case: also the causal pair")
+    ap.add_argument("--profile-d64", action="store_true",
+                    help="with --profile-case: d = 64 instead of 128 (B1 H64 N4096 d64, no 8-bit forward)")
     ap.add_argument("--profile-decode", action="store_true",
                     help="run only the small paged-decode profiling case (2 launches, B32) for ncu")
     args = ap.parse_args()
