@@ -254,10 +254,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int c4 = 0; c4 < 8; ++c4) {
             const float4 d4 = sD[8 * hh + c4];
             const int c = 32 * hh + 4 * c4;
-            pk[2 * c4] = pack_bf16x2(p[c + 0] * (__uint_as_float(dr[4 * c4 + 0]) - d4.x),
-                                     p[c + 1] * (__uint_as_float(dr[4 * c4 + 1]) - d4.y));
-            pk[2 * c4 + 1] = pack_bf16x2(p[c + 2] * (__uint_as_float(dr[4 * c4 + 2]) - d4.z),
-                                         p[c + 3] * (__uint_as_float(dr[4 * c4 + 3]) - d4.w));
+            // packed pairs: the same subtract-then-multiply roundings, half the instructions
+            const float2 lo = fmul2(make_float2(p[c + 0], p[c + 1]),
+                                    fsub2(make_float2(__uint_as_float(dr[4 * c4 + 0]), __uint_as_float(dr[4 * c4 + 1])),
+                                          make_float2(d4.x, d4.y)));
+            const float2 hi = fmul2(make_float2(p[c + 2], p[c + 3]),
+                                    fsub2(make_float2(__uint_as_float(dr[4 * c4 + 2]), __uint_as_float(dr[4 * c4 + 3])),
+                                          make_float2(d4.z, d4.w)));
+            pk[2 * c4] = pack_bf16x2(lo.x, lo.y);
+            pk[2 * c4 + 1] = pack_bf16x2(hi.x, hi.y);
           }
           tmem_st16(tR2 + 16 * hh, pk);
 #pragma unroll
