@@ -76,11 +76,15 @@ struct FwdShape {
 // about a fifth of the (query tile, key tile) steps, each a stall of the
 // softmax warps for a read-modify-write of O in TMEM.
 constexpr float kTau = 12.0f;
-// When > 0, one score pair in kPolyEvery takes its exponentials on the FMA pipe
-// (exp2_poly2) instead of the MUFU unit.  Measured on B200 at d = 128 the MUFU
-// is not what limits this kernel (1/4, 1/3 and 1/2 of the pairs on the FMA pipe
-// were 6-10% slower than none), so it is off.
-constexpr int kPolyEvery = 0;
+// When > 0, one score pair in kPolyEvery<D, kT> takes its exponentials on the FMA
+// pipe (exp2_poly2) instead of the MUFU unit.  Measured on B200 with the converged
+// MMA warp: at d = 64 with two query tiles per CTA, one pair in 8 is 3.5% faster
+// (B1 H32 N16384; 1% causal): the MMAs are half as long as at d = 128, so the two
+// softmax warpgroups' exponentials overlap more.  At d = 128 the same share cost
+// the bench step's forward 2%, and with one query tile per CTA (short walks) 13%,
+// so those instantiations keep every exponential on the MUFU unit.
+template <int D, int kT>
+constexpr int kPolyEvery = (D == 64 && kT == 2) ? 8 : 0;
 
 template <int D, int kT>
 struct FwdCfg {
@@ -328,7 +332,8 @@ __global__ void __launch_bounds__(FwdShape<kT>::kThreads, FwdShape<kT>::kMinBloc
             const float2 x = ffma2(make_float2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sl2v, negmv);
             float2 p = make_float2(0.f, 0.f);
             bool poly = false;
-            if constexpr (kPolyEvery > 0) poly = (i % (kPolyEvery > 0 ? kPolyEvery : 1)) == kPolyEvery - 1;
+            constexpr int kPoly = kPolyEvery<D, kT>;
+            if constexpr (kPoly > 0) poly = (i % (kPoly > 0 ? kPoly : 1)) == kPoly - 1;
             if (poly) {
               p = exp2_poly2(x);
             } else {
