@@ -60,10 +60,11 @@ struct FwdShape {
   static constexpr int kThreads = 128 * (kT + 1);
   static constexpr int kMinBlocks = (kT == 1) ? 2 : 1;
   // Register split (per thread): kT = 2: 384 x 168 at launch = 256 x 216 + 128 x 72;
-  // kT = 1: 256 x 128 = 128 x 192 + 128 x 64 (two CTAs share the register file).
+  // kT = 1: 256 x 128 = 128 x 208 + 128 x 48 (two CTAs share the register file;
+  // 192 for the softmax warps left it spilling).
   static constexpr uint32_t kRegLaunch = (kT == 1) ? 128 : 168;
-  static constexpr uint32_t kRegSoftmax = (kT == 1) ? 192 : 216;
-  static constexpr uint32_t kRegOther = (kT == 1) ? 64 : 72;
+  static constexpr uint32_t kRegSoftmax = (kT == 1) ? 208 : 216;
+  static constexpr uint32_t kRegOther = (kT == 1) ? 48 : 72;
   static constexpr uint32_t kTmemCols = (kT == 1) ? 256 : 512;
   static_assert(kRegSoftmax >= kRegLaunch && kRegOther <= kRegLaunch, "setmaxnreg direction");
   static_assert(kT * kRegSoftmax + kRegOther == (kT + 1) * kRegLaunch, "register split must match the launch");
